@@ -1,0 +1,129 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check the pins catch each.
+
+A pin set that passes a wrong oracle proves nothing; each mutation below is a
+mistake a reader could make from the block's definition, and at least one pin
+must fail on it.
+"""
+import math
+import types
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+from tests import oracle_pins as P
+from video_diffusion_vae_b200 import synth
+
+
+def _ns(**over):
+    d = {k: getattr(O, k) for k in ("silu", "norm_silu", "causal_conv3d", "causal_conv3d_at",
+                                    "upsample_nearest2x", "pixel_shuffle2x2", "resblock")}
+    d.update(over)
+    return types.SimpleNamespace(**d)
+
+
+def conv_flipped_time(x, wt, bias=None, cache=None, threads=None):
+    return O.causal_conv3d(x, np.ascontiguousarray(np.asarray(wt)[:, :, ::-1]), bias, cache, threads)
+
+
+def conv_centered_time(x, wt, bias=None, cache=None, threads=None):
+    # pads one frame on each side instead of two in front
+    x = np.asarray(x)
+    xp = np.concatenate([x[:, 1:], np.zeros_like(x[:, :1])], axis=1)
+    return O.causal_conv3d(xp, wt, bias, cache, threads)
+
+
+def conv_no_bias(x, wt, bias=None, cache=None, threads=None):
+    return O.causal_conv3d(x, wt, None, cache, threads)
+
+
+def conv_transposed_spatial(x, wt, bias=None, cache=None, threads=None):
+    return O.causal_conv3d(x, np.ascontiguousarray(np.swapaxes(np.asarray(wt), 3, 4)), bias, cache, threads)
+
+
+def norm_variance_eps(x, gamma, beta, eps=1e-12, apply_silu=True):
+    x = np.asarray(x, dtype=np.float64)
+    C = x.shape[0]
+    s = x / np.sqrt((x ** 2).mean(0, keepdims=True) + eps)
+    s = s * np.asarray(gamma).reshape((C,) + (1,) * (x.ndim - 1)) + np.asarray(beta).reshape((C,) + (1,) * (x.ndim - 1))
+    return s / (1 + np.exp(-s)) if apply_silu else s
+
+
+def norm_no_root_c(x, gamma, beta, eps=1e-12, apply_silu=True):
+    C = np.asarray(x).shape[0]
+    g = np.asarray(gamma, dtype=np.float64) / math.sqrt(C)
+    b = np.asarray(beta, dtype=np.float64)
+    return O.norm_silu(x, g, b, eps, apply_silu)
+
+
+def norm_sigmoid(x, gamma, beta, eps=1e-12, apply_silu=True):
+    s = O.norm_silu(x, gamma, beta, eps, False)
+    return 1 / (1 + np.exp(-s)) if apply_silu else s
+
+
+def silu_wrong(s):
+    return s / (1 + math.exp(s))
+
+
+def shuffle_swapped(x):
+    x = np.asarray(x)
+    C4 = x.shape[0]
+    idx = [4 * (k // 4) + 2 * (k % 2) + (k % 4) // 2 for k in range(C4)]
+    return O.pixel_shuffle2x2(x[idx])
+
+
+def upsample_bilinearish(x):
+    y = O.upsample_nearest2x(x)
+    y[:, :, 1::2] = 0.5 * (y[:, :, 1::2] + np.roll(y[:, :, 1::2], -1, axis=2))
+    return y
+
+
+def resblock_no_residual(x, p, threads=None):
+    return O.resblock(x, p, threads) - np.asarray(x, dtype=np.float64)
+
+
+def resblock_shortcut_on_normed(x, p, threads=None):
+    if p.get("ws") is None:
+        return O.resblock(x, p, threads)
+    a = O.norm_silu(x, p["gamma1"], p["beta1"])
+    h = O.causal_conv3d(O.norm_silu(O.causal_conv3d(a, p["w1"], p["b1"]), p["gamma2"], p["beta2"]),
+                        p["w2"], p["b2"])
+    return h + O.causal_conv3d(a, p["ws"], p["bs"])
+
+
+MUTANTS = {
+    "conv_flipped_time": _ns(causal_conv3d=conv_flipped_time),
+    "conv_centered_time": _ns(causal_conv3d=conv_centered_time),
+    "conv_no_bias": _ns(causal_conv3d=conv_no_bias),
+    "conv_transposed_spatial": _ns(causal_conv3d=conv_transposed_spatial),
+    "norm_variance_eps": _ns(norm_silu=norm_variance_eps),
+    "norm_no_root_c": _ns(norm_silu=norm_no_root_c),
+    "norm_sigmoid": _ns(norm_silu=norm_sigmoid),
+    "silu_wrong": _ns(silu=silu_wrong),
+    "shuffle_swapped": _ns(pixel_shuffle2x2=shuffle_swapped),
+    "upsample_blend": _ns(upsample_nearest2x=upsample_bilinearish),
+    "resblock_no_residual": _ns(resblock=resblock_no_residual),
+}
+
+
+def _fails(ns, extra=()):
+    for check in list(P.ALL_CHECKS) + list(extra):
+        try:
+            check(ns)
+        except AssertionError:
+            return True
+    return False
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name):
+    assert _fails(MUTANTS[name]), f"no pin failed for planted mistake {name}"
+
+
+def test_pins_catch_shortcut_on_normalised_input():
+    ns = _ns(resblock=resblock_shortcut_on_normed)
+    assert _fails(ns, extra=[lambda o: P.check_resblock_library(o, synth)])
+
+
+def test_real_oracle_passes_everything():
+    assert not _fails(O, extra=[lambda o: P.check_resblock_library(o, synth)])
