@@ -1,0 +1,195 @@
+/*
+ * wvae.h - C ABI of the B200 (sm_100a) Wan-style video-VAE decoder hot path.
+ *
+ * The operations are those of the Wan2.2 VAE decoder's residual block and the
+ * layers around it:
+ *   - channel RMS-norm + affine + SiLU ("Opt-in BF16 norm-SiLU fusion for Wan
+ *     VAE decoding", TensorRT-LLM issue #19309, section "Feature, motivation
+ *     and proposed scope": decoder residual norm1/norm2 and norm_out);
+ *   - causal 3x3x3 conv3d with bf16 operands and fp32 accumulation (FastVideo
+ *     "Wan2.2 VAE decoder (sm_100a, sm_103a)" README, section "Limits");
+ *   - the residual block, the nearest-2x upsample + 3x3 conv, and the decoder
+ *     trunk from latents [1, 48, T, H, W] to video [1, 3, T, 16H, 16W]
+ *     (same README, opening section: 48 latent channels, 16x16 spatial
+ *     compression; raw entry points are destination-passing on the current
+ *     stream, section "Use").
+ *
+ * Conventions shared by every entry point:
+ *   - Memory: every pointer argument named as a tensor is a DEVICE pointer owned
+ *     by the caller; the library never allocates, frees or keeps device memory
+ *     (the only device-side state is a 4-byte error word, see
+ *     wvae_device_error).  Arrays of pointers (wvae_decode_trunk) are HOST
+ *     arrays holding device pointers.
+ *   - Layout: activations are batch-1 channels-last [T][H][W][C], contiguous.
+ *     The trunk alone takes its latents and returns its video in NCDHW order
+ *     ([1][C][T][H][W]) as the FastVideo decoder does.
+ *   - Streams: work is enqueued on `stream` (NULL = legacy default stream) and
+ *     the call returns without synchronising.  No call blocks on the device.
+ *   - Errors: arguments are validated on the host before anything is launched;
+ *     a failed check returns a non-zero wvae_status and enqueues nothing.  A
+ *     launch failure returns WVAE_ERR_CUDA.  Device-side faults detected by
+ *     the kernels (a pipeline wait that exceeded its time limit) are recorded
+ *     in the error word and reported by wvae_device_error.
+ *   - dtype WVAE_BF16: bf16 activations and weights, fp32 accumulation and
+ *     fp32 norm statistics, tensor cores (tcgen05).  WVAE_F32: fp32 storage
+ *     and CUDA-core fp32 arithmetic (a precision reference path).
+ *   - Pointers must be 16-byte aligned.  In-place operation is allowed only
+ *     where stated.
+ */
+#ifndef WVAE_H
+#define WVAE_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define WVAE_API __attribute__((visibility("default")))
+#else
+#define WVAE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* wvae_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  WVAE_OK = 0,
+  WVAE_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, mismatch      */
+  WVAE_ERR_UNSUPPORTED = 2,  /* shape/dtype outside what the kernels handle     */
+  WVAE_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned                */
+  WVAE_ERR_WORKSPACE = 4,    /* workspace / packed buffer smaller than required */
+  WVAE_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed            */
+  WVAE_ERR_TIMEOUT = 6,      /* a kernel wait exceeded its limit (device word)  */
+  WVAE_ERR_NO_DEVICE = 7     /* no sm_100 device is current                     */
+} wvae_status;
+
+typedef enum { WVAE_BF16 = 0, WVAE_F32 = 1 } wvae_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+WVAE_API const char* wvae_status_string(int status);
+
+/* ABI version: (major << 16) | minor. */
+WVAE_API int wvae_version(void);
+
+/*
+ * Device error word: returns WVAE_OK if no kernel since the last reset has
+ * recorded a fault, else WVAE_ERR_TIMEOUT; *code (may be NULL) receives the raw
+ * bit mask.  Synchronises the current device.  reset != 0 clears the word.
+ */
+WVAE_API wvae_status wvae_device_error(unsigned int* code, int reset);
+
+/* ---------------------------------------------------------------- norm-SiLU
+ * Channel RMS-norm + affine + SiLU at every voxel v of x [T][H][W][C]:
+ *   y[v,c] = SiLU( x[v,c] / max(||x[v,:]||_2, eps) * sqrt(C) * gamma[c] + beta[c] )
+ * with SiLU(s) = s / (1 + exp(-s)); statistics in fp32.
+ * (TensorRT-LLM issue #19309, "Feature, motivation and proposed scope";
+ * FastVideo README "Limits": fp32 RMS-norm statistics.)
+ *   x, y     : [T*H*W][C] in `dtype`; y may equal x (in place).
+ *   gamma, beta : fp32 [C].
+ *   C        : multiple of 8 (bf16) / 4 (fp32), 8 <= C <= 1024.
+ *   eps      : > 0 (the decoder uses 1e-12).
+ */
+WVAE_API wvae_status wvae_norm_silu(const void* x, void* y, const float* gamma, const float* beta,
+                           int T, int H, int W, int C, float eps, wvae_dtype dtype,
+                           wvae_stream_t stream);
+
+/* ------------------------------------------------------------ weight prepack
+ * One-time re-layout of a conv's weights into the tile order the conv kernels
+ * read (FastVideo README, "Use": the decoder prepares its weights once).
+ * Source: PyTorch order [cout][cin][kt][kh][kw] (fp32 if w_dtype == WVAE_F32,
+ * bf16 if WVAE_BF16), device memory; bias fp32 [cout] or NULL (zero).
+ * `dtype` selects the compute path the packed blob is for.  The blob is
+ * opaque, position-independent and owned by the caller; it can be copied or
+ * saved as bytes.  Supported kernel sizes: (3,3,3), (1,3,3), (1,1,1).
+ * wvae_conv_packed_bytes returns 0 for unsupported shapes.
+ */
+WVAE_API size_t wvae_conv_packed_bytes(int cout, int cin, int kt, int kh, int kw, wvae_dtype dtype);
+WVAE_API wvae_status wvae_prepack_conv(const void* w, wvae_dtype w_dtype, const float* bias, int cout,
+                              int cin, int kt, int kh, int kw, wvae_dtype dtype, void* packed,
+                              size_t packed_bytes, wvae_stream_t stream);
+
+/* ------------------------------------------------------------ causal conv3d
+ * out[t,h,w,o] = bias[o] + sum_{i,kt,kh,kw} W[o,i,kt,kh,kw] * a[t+kt-(KT-1), h+kh-(KH-1)/2,
+ *                                                              w+kw-(KW-1)/2, i]
+ * where a = x (or SiLU(norm(x)) when norm_gamma/norm_beta are given), zero
+ * outside [0,H)x[0,W), and for frames t' < 0 the previous chunk's frame
+ * cache[KT-1+t'] when `cache` is given, else zero (two zero frames in front
+ * for KT = 3).  Padding applies after the norm: padded inputs are exactly 0.
+ * Optionally out += residual (same layout as y).
+ *   x        : [T][H][W][cin] in dtype.   cache: NULL or [KT-1][H][W][cin]
+ *              holding the previous chunk's conv INPUT (already normalised).
+ *   packed_w : from wvae_prepack_conv for (cout, cin, kt, kh, kw, dtype).
+ *   norm_gamma, norm_beta : both NULL (no norm) or both fp32 [cin]; eps 1e-12.
+ *   residual : NULL or [T][H][W][cout] in dtype.   y: [T][H][W][cout].
+ *   workspace: wvae_causal_conv3d_workspace_bytes(...) bytes (0 without norm).
+ * bf16: cin % 64 == 0, cout % 16 == 0 and cout <= 256 or cout == 512.
+ * y must not overlap x, cache or residual.
+ */
+WVAE_API size_t wvae_causal_conv3d_workspace_bytes(int T, int H, int W, int cin, int has_norm,
+                                          wvae_dtype dtype);
+WVAE_API wvae_status wvae_causal_conv3d(const void* x, const void* cache, const void* packed_w, int T,
+                               int H, int W, int cin, int cout, int kt, int kh, int kw,
+                               const float* norm_gamma, const float* norm_beta,
+                               const void* residual, void* y, wvae_dtype dtype, void* workspace,
+                               size_t ws_bytes, wvae_stream_t stream);
+
+/* ------------------------------------------------------------ residual block
+ * h = shortcut(x) + conv2(A2(conv1(A1(x)))), A_k = SiLU(norm_k(.)), causal
+ * 3x3x3 convs; shortcut = identity when cin == cout, else the 1x1x1 conv
+ * packed in wsc_packed (applied to the raw x).  The norm of conv1's output is
+ * computed in conv1's epilogue and the shortcut is folded into conv2's
+ * reduction, so the block is 3 kernels (norm1, conv1, conv2).
+ *   x: [T][H][W][cin], y: [T][H][W][cout] in dtype (y must not overlap x).
+ *   w1_packed (cout, cin, 3,3,3), w2_packed (cout, cout, 3,3,3),
+ *   wsc_packed (cout, cin, 1,1,1) or NULL iff cin == cout.
+ *   gamma1/beta1 fp32 [cin], gamma2/beta2 fp32 [cout].
+ *   workspace: wvae_resblock_workspace_bytes(...) bytes.
+ */
+WVAE_API size_t wvae_resblock_workspace_bytes(int T, int H, int W, int cin, int cout, wvae_dtype dtype);
+WVAE_API wvae_status wvae_resblock(const void* x, void* y, int T, int H, int W, int cin, int cout,
+                          const float* gamma1, const float* beta1, const void* w1_packed,
+                          const float* gamma2, const float* beta2, const void* w2_packed,
+                          const void* wsc_packed, wvae_dtype dtype, void* workspace,
+                          size_t ws_bytes, wvae_stream_t stream);
+
+/* -------------------------------------------------- upsample + 3x3 conv
+ * y[t] = conv3x3( nearest2x(x[t]) ) + bias, per frame, zero border of 1 at the
+ * upsampled resolution; u[2h+i, 2w+j] = x[h, w].
+ *   x: [T][H][W][cin], y: [T][2H][2W][cout] in dtype.
+ *   packed_w: (cout, cin, 1, 3, 3).   workspace: see the _bytes query.
+ */
+WVAE_API size_t wvae_upsample_conv_workspace_bytes(int T, int H, int W, int cin, wvae_dtype dtype);
+WVAE_API wvae_status wvae_upsample_conv(const void* x, void* y, int T, int H, int W, int cin, int cout,
+                               const void* packed_w, wvae_dtype dtype, void* workspace,
+                               size_t ws_bytes, wvae_stream_t stream);
+
+/* ------------------------------------------------------------ decoder trunk
+ * Wan2.2-shaped decoder trunk on latents z [1][48][T][H][W] (NCDHW, bf16):
+ *   conv_in (causal 3x3x3, 48 -> C0)
+ *   stage s = 0..3 at resolution (2^s H, 2^s W): 2 residual blocks of width Cs,
+ *     then for s < 3 a nearest-2x upsample + 3x3 conv Cs -> C(s+1)
+ *   norm_out + SiLU, causal 3x3x3 conv C3 -> 12, 2x2 pixel shuffle
+ *   -> video [1][3][T][16H][16W] (NCDHW, bf16), video[c,t,2h+i,2w+j] = out[4c+2i+j].
+ *   widths: host int[4] (C0..C3), NULL = {512, 512, 256, 128}; each a multiple of
+ *     64 and <= 256 or == 512.
+ *   packed: host array of 21 device pointers, in forward order:
+ *     [0] conv_in (C0, 48, 3,3,3); per stage s, per block b: conv1 (Cs, Cs, 3,3,3),
+ *     conv2 (Cs, Cs, 3,3,3); then for s < 3 the upsample conv (C(s+1), Cs, 1,3,3);
+ *     [20] head (12, C3, 3,3,3).
+ *   norms: host array of 34 device pointers (fp32), gamma then beta for each norm in
+ *     forward order: per stage, per block: norm1, norm2; then norm_out.
+ *   workspace: wvae_decode_trunk_workspace_bytes(T, H, W, widths) bytes.
+ * Only dtype == WVAE_BF16 is supported.
+ */
+WVAE_API size_t wvae_decode_trunk_workspace_bytes(int T, int H, int W, const int* widths);
+WVAE_API wvae_status wvae_decode_trunk(const void* const* packed, const float* const* norms,
+                              const void* z, void* video, int T, int H, int W, const int* widths,
+                              wvae_dtype dtype, void* workspace, size_t ws_bytes,
+                              wvae_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* WVAE_H */

@@ -1,0 +1,90 @@
+"""Causal conv3d (tcgen05 implicit GEMM and the fp32 path) vs the oracle (GPU)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from tests.gpu_util import assert_close, from_cl, sample_voxels, to_cl
+from video_diffusion_vae_b200 import binding as B
+from video_diffusion_vae_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(x, w, b, dtype, **kw):
+    pk = B.prepack_conv(w.cuda().to(dtype), b.cuda(), dtype)
+    return pk, B.causal_conv3d(to_cl(x, dtype), pk, **kw)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_conv_tiny_config(dtype):
+    """Config 0's conv: 64 -> 64, x [64, 2, 16, 16]."""
+    x, w, b = synth.conv_input(cin=64, cout=64, T=2, H=16, W=16, seed=0, bf16=dtype == torch.bfloat16)
+    _, y = _run(x, w, b, dtype)
+    assert_close(from_cl(y), O.causal_conv3d(x, w, b), dtype, "tiny")
+
+
+@pytest.mark.parametrize("cout", [16, 64, 128, 256, 512])
+def test_conv_ragged_tiles(cout):
+    """H, W not multiples of the 8 x 16 tile; T = 3; several output widths."""
+    x, w, b = synth.conv_input(cin=64, cout=cout, T=3, H=13, W=21, seed=cout)
+    _, y = _run(x, w, b, torch.bfloat16)
+    assert_close(from_cl(y), O.causal_conv3d(x, w, b), torch.bfloat16, f"cout={cout}")
+
+
+@pytest.mark.parametrize("k", [(1, 3, 3), (1, 1, 1), (3, 3, 3)])
+def test_conv_kernel_sizes_two_chunks(k):
+    x, w, b = synth.conv_input(cin=128, cout=64, T=2, H=9, W=17, seed=7, k=k)
+    _, y = _run(x, w, b, torch.bfloat16)
+    assert_close(from_cl(y), O.causal_conv3d(x, w, b), torch.bfloat16, f"k={k}")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_conv_with_residual_norm_and_cache(dtype):
+    bf = dtype == torch.bfloat16
+    x, w, b = synth.conv_input(cin=64, cout=64, T=3, H=10, W=18, seed=11, bf16=bf)
+    g = torch.Generator().manual_seed(12)
+    res = torch.randn(64, 3, 10, 18, generator=g)
+    res = res.to(torch.bfloat16).float() if bf else res
+    gamma = 1 + 0.3 * torch.randn(64, generator=g)
+    beta = 0.3 * torch.randn(64, generator=g)
+    cache = torch.randn(64, 2, 10, 18, generator=g)
+    cache = cache.to(torch.bfloat16).float() if bf else cache
+    pk = B.prepack_conv(w.cuda().to(dtype), b.cuda(), dtype)
+    # residual
+    y = B.causal_conv3d(to_cl(x, dtype), pk, residual=to_cl(res, dtype))
+    assert_close(from_cl(y), O.causal_conv3d(x, w, b) + res.double().numpy(), dtype, "residual")
+    # norm + SiLU before the conv (padding applies after the norm)
+    y = B.causal_conv3d(to_cl(x, dtype), pk, norm=(gamma.cuda(), beta.cuda()))
+    ref = O.causal_conv3d(O.norm_silu(x, gamma, beta), w, b)
+    assert_close(from_cl(y), ref, dtype, "norm")
+    # previous chunk's cached frames in place of the zero frames
+    y = B.causal_conv3d(to_cl(x, dtype), pk, cache=to_cl(cache, dtype))
+    assert_close(from_cl(y), O.causal_conv3d(x, w, b, cache=cache), dtype, "cache")
+
+
+def test_conv_causality_bitwise():
+    """Changing frame t leaves every output frame before t bit-identical."""
+    x, w, b = synth.conv_input(cin=64, cout=128, T=4, H=9, W=20, seed=13)
+    pk = B.prepack_conv(w.cuda().bfloat16(), b.cuda())
+    y0 = B.causal_conv3d(to_cl(x), pk)
+    x2 = x.clone()
+    x2[:, 2] = torch.randn(64, 9, 20, generator=torch.Generator().manual_seed(14)).bfloat16().float()
+    y1 = B.causal_conv3d(to_cl(x2), pk)
+    assert torch.equal(y0[:2], y1[:2])
+    assert not torch.equal(y0[2], y1[2])
+
+
+def test_conv_full_size_sampled():
+    """Config 2: 512 -> 512 on [512, 4, 88, 156]; sampled voxels against the oracle."""
+    x, w, b = synth.conv_input(cin=512, cout=512, T=4, H=88, W=156, seed=0)
+    pk = B.prepack_conv(w.cuda().bfloat16(), b.cuda())
+    y = B.causal_conv3d(to_cl(x), pk)
+    torch.cuda.synchronize()
+    yc = y.float().cpu()
+    pts = sample_voxels(4, 88, 156, 48, seed=2)
+    got = np.stack([yc[t, h, ww].double().numpy() for (t, h, ww) in pts], 1)
+    ref = np.stack([O.causal_conv3d_at(x, w, b, t, h, ww) for (t, h, ww) in pts], 1)
+    assert_close(got, ref, torch.bfloat16, "config 2 sampled")
+    assert torch.isfinite(yc).all()
+    assert B.device_error() == 0

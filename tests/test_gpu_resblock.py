@@ -1,0 +1,104 @@
+"""Residual block, upsample conv and decoder trunk vs the oracle (GPU)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from tests.gpu_util import assert_close, from_cl, sample_voxels, to_cl
+from video_diffusion_vae_b200 import binding as B
+from video_diffusion_vae_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def resblock_at(x, p, t, h, w):
+    """Oracle block output at one voxel from the crop that determines it: frames
+    t-4..t and a 2-pixel border (two stacked causal 3x3x3 convs).  Where the crop
+    meets the tensor's edge the zero padding is the real one; elsewhere the
+    crop's own padding only reaches outputs that are not read."""
+    _, T, H, W = x.shape
+    t0, h0, h1, w0, w1 = max(0, t - 4), max(0, h - 2), min(H, h + 3), max(0, w - 2), min(W, w + 3)
+    y = O.resblock(x[:, t0:t + 1, h0:h1, w0:w1], p, threads=8)
+    return y[:, t - t0, h - h0, w - w0]
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_resblock_tiny_config(dtype):
+    """Config 0: x [64, 2, 16, 16], two (norm + SiLU + conv 64->64) stages + identity."""
+    x, p = synth.tiny_resblock(bf16=dtype == torch.bfloat16)
+    blk = B.PackedResBlock(p, dtype)
+    y = B.resblock(to_cl(x, dtype), blk)
+    assert_close(from_cl(y), O.resblock(x, p), dtype, "config 0")
+
+
+@pytest.mark.parametrize("cin,cout", [(256, 256), (256, 128), (128, 64), (64, 128)])
+def test_resblock_reduced(cin, cout):
+    x, p = synth.resblock_input(cin=cin, cout=cout, T=3, H=11, W=19, seed=cin + cout)
+    blk = B.PackedResBlock(p)
+    y = B.resblock(to_cl(x), blk)
+    assert_close(from_cl(y), O.resblock(x, p), torch.bfloat16, f"{cin}->{cout}")
+
+
+@pytest.mark.parametrize("cout", [256, 128])
+def test_resblock_full_size_sampled(cout):
+    """Config 3 (and its 256 -> 128 shortcut variant) at [256, 4, 176, 312]."""
+    x, p = synth.resblock_input(cin=256, cout=cout, T=4, H=176, W=312, seed=0)
+    blk = B.PackedResBlock(p)
+    y = B.resblock(to_cl(x), blk)
+    torch.cuda.synchronize()
+    yc = y.float().cpu()
+    pts = sample_voxels(4, 176, 312, 12, seed=3)
+    got = np.stack([yc[t, h, w].double().numpy() for (t, h, w) in pts], 1)
+    ref = np.stack([resblock_at(x, p, t, h, w) for (t, h, w) in pts], 1)
+    assert_close(got, ref, torch.bfloat16, f"config 3 cout={cout}")
+    assert torch.isfinite(yc).all()
+    assert B.device_error() == 0
+
+
+@pytest.mark.parametrize("cin,cout,H,W", [(128, 64, 6, 10), (64, 128, 5, 9), (512, 256, 4, 8)])
+def test_upsample_conv(cin, cout, H, W):
+    g = torch.Generator().manual_seed(cin)
+    x = synth.normal(g, (cin, 2, H, W))
+    w, b = synth.conv_params(g, cout, cin, 1, 3, 3)
+    pk = B.prepack_conv(w.cuda().bfloat16(), b.cuda())
+    y = B.upsample_conv(to_cl(x), pk)
+    assert_close(from_cl(y), O.upsample_conv(x, w, b), torch.bfloat16, "upsample conv")
+
+
+def _trunk_case(T, H, W, widths, zc=48, seed=0):
+    z, params = synth.trunk_input(T=T, H=H, W=W, widths=widths, zc=zc, seed=seed)
+    tr = B.PackedTrunk(params)
+    video = B.decode_trunk(z[None].cuda().bfloat16().contiguous(), tr)
+    return z, params, video
+
+
+def test_trunk_reduced_width_end_to_end():
+    z, params, video = _trunk_case(T=3, H=3, W=5, widths=(128, 128, 64, 64))
+    assert video.shape == (1, 3, 3, 48, 80)
+    ref = O.trunk(z, params)
+    assert_close(video[0].float().cpu().double().numpy(), ref, torch.bfloat16, "trunk reduced")
+
+
+@pytest.mark.slow
+def test_trunk_full_width_end_to_end():
+    z, params, video = _trunk_case(T=2, H=4, W=6, widths=synth.TRUNK_WIDTHS)
+    ref = O.trunk(z, params)
+    assert_close(video[0].float().cpu().double().numpy(), ref, torch.bfloat16, "trunk full width")
+
+
+def test_trunk_full_size_properties():
+    """Config 4 at full size: finite, deterministic, and causal bit for bit."""
+    z, params = synth.trunk_input(T=4, H=44, W=78, seed=0)
+    tr = B.PackedTrunk(params)
+    zd = z[None].cuda().bfloat16().contiguous()
+    v0 = B.decode_trunk(zd, tr)
+    v1 = B.decode_trunk(zd, tr)
+    assert v0.shape == (1, 3, 4, 704, 1248)
+    assert torch.isfinite(v0.float()).all()
+    assert torch.equal(v0, v1)
+    z2 = zd.clone()
+    z2[:, :, 3] = torch.randn(1, 48, 44, 78, generator=torch.Generator().manual_seed(9)).bfloat16().cuda()
+    v2 = B.decode_trunk(z2, tr)
+    assert torch.equal(v0[:, :, :3], v2[:, :, :3])
+    assert not torch.equal(v0[:, :, 3], v2[:, :, 3])
+    assert B.device_error() == 0

@@ -1,0 +1,677 @@
+// The exported C ABI (include/wvae.h): argument validation, TMA descriptors,
+// conv planning and the composition of the residual block, the upsample conv
+// and the decoder trunk out of the kernels.  Nothing here allocates device
+// memory: every buffer, including workspaces, belongs to the caller.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/wvae.h"
+#include "internal.h"
+
+namespace wvae {
+
+__device__ unsigned g_device_error = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool init = false;
+  bool ok = false;
+  int num_sms = 0;
+  unsigned* err = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+wvae_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return WVAE_ERR_NO_DEVICE;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    d.init = true;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return WVAE_ERR_NO_DEVICE;
+    }
+    void* sym = nullptr;
+    if (major == 10 && minor == 0 && cudaGetSymbolAddress(&sym, g_device_error) == cudaSuccess) {
+      d.err = static_cast<unsigned*>(sym);
+      d.ok = true;
+    }
+    cudaGetLastError();
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+              cudaSuccess &&
+          q == cudaDriverEntryPointSuccess)
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+      cudaGetLastError();
+    }
+  }
+  if (!d.ok || g_encode == nullptr) return WVAE_ERR_NO_DEVICE;
+  *out = &d;
+  return WVAE_OK;
+}
+
+inline bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
+inline size_t round_up_sz(size_t v, size_t m) { return (v + m - 1) / m * m; }
+
+inline wvae_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return WVAE_OK;
+  cudaGetLastError();
+  return WVAE_ERR_CUDA;
+}
+
+bool kernel_ok(int kt, int kh, int kw) {
+  return (kt == 3 && kh == 3 && kw == 3) || (kt == 1 && kh == 3 && kw == 3) ||
+         (kt == 1 && kh == 1 && kw == 1);
+}
+
+// --------------------------------------------------------- packed weights
+struct PackedLayout {
+  int cout_pad, cin_pad, taps;
+  size_t w_bytes, bias_off, total;
+};
+
+PackedLayout packed_layout(int cout, int cin, int kt, int kh, int kw, wvae_dtype dtype) {
+  PackedLayout L;
+  L.taps = kt * kh * kw;
+  if (dtype == WVAE_BF16) {
+    L.cout_pad = round_up(cout, 16);
+    L.cin_pad = round_up(cin, 64);
+    L.w_bytes = static_cast<size_t>(L.cout_pad) * L.taps * L.cin_pad * 2;
+  } else {
+    L.cout_pad = cout;
+    L.cin_pad = cin;
+    L.w_bytes = static_cast<size_t>(cout) * L.taps * cin * 4;
+  }
+  L.bias_off = round_up_sz(L.w_bytes, 256);
+  L.total = L.bias_off + static_cast<size_t>(L.cout_pad) * 4;
+  return L;
+}
+
+// ------------------------------------------------------------ TMA descriptors
+bool encode_act(CUtensorMap* m, const void* base, int C, int W, int H, int T) {
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(W),
+                        static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(C) * 2, static_cast<cuuint64_t>(C) * 2 * W,
+                           static_cast<cuuint64_t>(C) * 2 * W * H};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(kTileW),
+                       static_cast<cuuint32_t>(kTileH), 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+bool encode_weights(CUtensorMap* m, const void* base, int K, int N, int box_rows) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t es[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// --------------------------------------------------------- tensor-core conv
+struct TcConv {
+  const void* x = nullptr;   // [T][H][W][cin_pad] bf16
+  int cin_pad = 0;
+  const void* cache = nullptr;
+  const void* packed = nullptr;
+  int cout = 0, KT = 3, KH = 3, KW = 3;
+  const void* x2 = nullptr;  // shortcut input [T][H][W][cin2_pad]
+  int cin2_pad = 0;
+  const void* packed2 = nullptr;
+  int T = 0, H = 0, W = 0;
+  ConvEpilogue ep{};
+};
+
+wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
+  static_assert(sizeof(ConvParams) < 4000, "kernel parameter space");
+  const PackedLayout L = packed_layout(a.cout, a.cin_pad, a.KT, a.KH, a.KW, WVAE_BF16);
+  ConvParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.T = a.T;
+  p.H = a.H;
+  p.W = a.W;
+  p.cin_pad = a.cin_pad;
+  p.cin2_pad = a.cin2_pad;
+  p.cout = a.cout;
+  p.cout_pad = L.cout_pad;
+  p.KT = a.KT;
+  p.KH = a.KH;
+  p.KW = a.KW;
+  p.has_cache = a.cache != nullptr;
+  const bool need_all_channels = a.ep.act != nullptr;
+  if (L.cout_pad <= 256) {
+    p.BN = L.cout_pad;
+  } else if (L.cout_pad == 512) {
+    p.BN = need_all_channels ? 512 : 256;
+  } else {
+    if (need_all_channels) return WVAE_ERR_UNSUPPORTED;
+    p.BN = (L.cout_pad % 256 == 0) ? 256 : (L.cout_pad % 128 == 0 ? 128 : 16);
+  }
+  p.n_tiles = L.cout_pad / p.BN;
+  p.num_acc = p.BN <= 256 ? 2 : 1;
+  p.stages = conv_tc_stages_for(p.BN);
+  p.tiles_w = (a.W + kTileW - 1) / kTileW;
+  p.tiles_h = (a.H + kTileH - 1) / kTileH;
+  p.m_tiles = a.T * p.tiles_h * p.tiles_w;
+  p.num_tiles = p.m_tiles * p.n_tiles;
+  p.kblocks_main = L.taps * (a.cin_pad / kBK);
+  p.kblocks = p.kblocks_main + a.cin2_pad / kBK;
+  a.ep.bias = reinterpret_cast<const float*>(static_cast<const char*>(a.packed) + L.bias_off);
+  if (a.packed2 != nullptr) {
+    const PackedLayout L2 = packed_layout(a.cout, a.cin2_pad, 1, 1, 1, WVAE_BF16);
+    a.ep.bias2 = reinterpret_cast<const float*>(static_cast<const char*>(a.packed2) + L2.bias_off);
+  }
+  p.ep = a.ep;
+  p.err = d.err;
+  const int box_rows = p.BN > 256 ? 256 : p.BN;
+  if (!encode_act(&p.tmA, a.x, a.cin_pad, a.W, a.H, a.T)) return WVAE_ERR_CUDA;
+  if (!encode_weights(&p.tmB, a.packed, L.taps * a.cin_pad, L.cout_pad, box_rows))
+    return WVAE_ERR_CUDA;
+  if (a.cache != nullptr && !encode_act(&p.tmC, a.cache, a.cin_pad, a.W, a.H, a.KT - 1))
+    return WVAE_ERR_CUDA;
+  if (a.cin2_pad > 0) {
+    if (!encode_act(&p.tmA2, a.x2, a.cin2_pad, a.W, a.H, a.T)) return WVAE_ERR_CUDA;
+    if (!encode_weights(&p.tmB2, a.packed2, a.cin2_pad, L.cout_pad, box_rows)) return WVAE_ERR_CUDA;
+  }
+  const int grid = p.num_tiles < d.num_sms ? p.num_tiles : d.num_sms;
+  return cuda_status(launch_conv_tc(p, grid, stream));
+}
+
+size_t bytes_of(wvae_dtype dt) { return dt == WVAE_BF16 ? 2 : 4; }
+
+bool bf16_cout_ok(int cout) { return cout > 0 && cout % 16 == 0 && (cout <= 256 || cout == 512); }
+
+}  // namespace
+
+unsigned* device_error_word() {
+  DeviceInfo* d = nullptr;
+  return device_info(&d) == WVAE_OK ? d->err : nullptr;
+}
+
+}  // namespace wvae
+
+using namespace wvae;
+
+extern "C" {
+
+const char* wvae_status_string(int status) {
+  switch (status) {
+    case WVAE_OK: return "ok";
+    case WVAE_ERR_INVALID_ARG: return "invalid argument";
+    case WVAE_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case WVAE_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case WVAE_ERR_WORKSPACE: return "workspace or packed buffer too small";
+    case WVAE_ERR_CUDA: return "CUDA error";
+    case WVAE_ERR_TIMEOUT: return "a kernel wait exceeded its limit";
+    case WVAE_ERR_NO_DEVICE: return "no sm_100 device is current";
+    default: return "unknown status";
+  }
+}
+
+int wvae_version(void) { return (1 << 16) | 0; }
+
+wvae_status wvae_device_error(unsigned int* code, int reset) {
+  DeviceInfo* d = nullptr;
+  wvae_status st = device_info(&d);
+  if (st != WVAE_OK) return st;
+  unsigned v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return cuda_status(cudaGetLastError());
+  if (cudaMemcpy(&v, d->err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return cuda_status(cudaGetLastError());
+  if (reset) {
+    const unsigned zero = 0;
+    if (cudaMemcpy(d->err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return cuda_status(cudaGetLastError());
+  }
+  if (code) *code = v;
+  return v ? WVAE_ERR_TIMEOUT : WVAE_OK;
+}
+
+// ------------------------------------------------------------------ norm-SiLU
+wvae_status wvae_norm_silu(const void* x, void* y, const float* gamma, const float* beta, int T,
+                           int H, int W, int C, float eps, wvae_dtype dtype, wvae_stream_t stream) {
+  if (!x || !y || !gamma || !beta) return WVAE_ERR_INVALID_ARG;
+  if (T < 1 || H < 1 || W < 1 || C < 1 || !(eps > 0.0f)) return WVAE_ERR_INVALID_ARG;
+  if (dtype != WVAE_BF16 && dtype != WVAE_F32) return WVAE_ERR_UNSUPPORTED;
+  const int vec = dtype == WVAE_BF16 ? 8 : 4;
+  if (C % vec != 0 || C < 8 || C > 1024) return WVAE_ERR_UNSUPPORTED;
+  if (!a16(x) || !a16(y)) return WVAE_ERR_ALIGNMENT;
+  DeviceInfo* d = nullptr;
+  wvae_status st = device_info(&d);
+  if (st != WVAE_OK) return st;
+  const long nvox = static_cast<long>(T) * H * W;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == WVAE_BF16)
+    return cuda_status(launch_norm_silu_bf16(static_cast<const __nv_bfloat16*>(x),
+                                             static_cast<__nv_bfloat16*>(y), gamma, beta, nvox, C,
+                                             eps, d->num_sms, s));
+  return cuda_status(launch_norm_silu_f32(static_cast<const float*>(x), static_cast<float*>(y),
+                                          gamma, beta, nvox, C, eps, d->num_sms, s));
+}
+
+// ------------------------------------------------------------------ prepack
+size_t wvae_conv_packed_bytes(int cout, int cin, int kt, int kh, int kw, wvae_dtype dtype) {
+  if (cout < 1 || cin < 1 || !kernel_ok(kt, kh, kw)) return 0;
+  if (dtype != WVAE_BF16 && dtype != WVAE_F32) return 0;
+  return packed_layout(cout, cin, kt, kh, kw, dtype).total;
+}
+
+wvae_status wvae_prepack_conv(const void* w, wvae_dtype w_dtype, const float* bias, int cout,
+                              int cin, int kt, int kh, int kw, wvae_dtype dtype, void* packed,
+                              size_t packed_bytes, wvae_stream_t stream) {
+  if (!w || !packed) return WVAE_ERR_INVALID_ARG;
+  if (cout < 1 || cin < 1) return WVAE_ERR_INVALID_ARG;
+  if (!kernel_ok(kt, kh, kw)) return WVAE_ERR_UNSUPPORTED;
+  if ((w_dtype != WVAE_BF16 && w_dtype != WVAE_F32) || (dtype != WVAE_BF16 && dtype != WVAE_F32))
+    return WVAE_ERR_UNSUPPORTED;
+  if (!a16(packed)) return WVAE_ERR_ALIGNMENT;
+  const PackedLayout L = packed_layout(cout, cin, kt, kh, kw, dtype);
+  if (packed_bytes < L.total) return WVAE_ERR_WORKSPACE;
+  DeviceInfo* d = nullptr;
+  wvae_status st = device_info(&d);
+  if (st != WVAE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* bias_p = reinterpret_cast<float*>(static_cast<char*>(packed) + L.bias_off);
+  if (dtype == WVAE_BF16)
+    return cuda_status(launch_prepack_bf16(w, w_dtype == WVAE_F32, bias, cout, cin, L.taps,
+                                           L.cout_pad, L.cin_pad,
+                                           static_cast<__nv_bfloat16*>(packed), bias_p, s));
+  return cuda_status(launch_prepack_f32(w, w_dtype == WVAE_F32, bias, cout, cin, L.taps,
+                                        static_cast<float*>(packed), bias_p, s));
+}
+
+// ------------------------------------------------------------- causal conv3d
+size_t wvae_causal_conv3d_workspace_bytes(int T, int H, int W, int cin, int has_norm,
+                                          wvae_dtype dtype) {
+  if (!has_norm || T < 1 || H < 1 || W < 1 || cin < 1) return 0;
+  return round_up_sz(static_cast<size_t>(T) * H * W * cin * bytes_of(dtype), 256);
+}
+
+wvae_status wvae_causal_conv3d(const void* x, const void* cache, const void* packed_w, int T,
+                               int H, int W, int cin, int cout, int kt, int kh, int kw,
+                               const float* norm_gamma, const float* norm_beta,
+                               const void* residual, void* y, wvae_dtype dtype, void* workspace,
+                               size_t ws_bytes, wvae_stream_t stream) {
+  if (!x || !packed_w || !y) return WVAE_ERR_INVALID_ARG;
+  if (T < 1 || H < 1 || W < 1 || cin < 1 || cout < 1) return WVAE_ERR_INVALID_ARG;
+  if ((norm_gamma == nullptr) != (norm_beta == nullptr)) return WVAE_ERR_INVALID_ARG;
+  if (!kernel_ok(kt, kh, kw)) return WVAE_ERR_UNSUPPORTED;
+  if (dtype != WVAE_BF16 && dtype != WVAE_F32) return WVAE_ERR_UNSUPPORTED;
+  if (cache != nullptr && kt < 2) return WVAE_ERR_INVALID_ARG;
+  if (x == y || (residual != nullptr && residual == y) || (cache != nullptr && cache == y))
+    return WVAE_ERR_INVALID_ARG;
+  if (!a16(x) || !a16(y) || !a16(packed_w) || (cache && !a16(cache)) ||
+      (residual && !a16(residual)) || (workspace && !a16(workspace)))
+    return WVAE_ERR_ALIGNMENT;
+  if (dtype == WVAE_BF16 && (cin % 64 != 0 || !bf16_cout_ok(cout))) return WVAE_ERR_UNSUPPORTED;
+  if (dtype == WVAE_F32 && (cin % 4 != 0 || cout % 4 != 0)) return WVAE_ERR_UNSUPPORTED;
+  const bool has_norm = norm_gamma != nullptr;
+  const size_t need = wvae_causal_conv3d_workspace_bytes(T, H, W, cin, has_norm, dtype);
+  if (has_norm && (workspace == nullptr || ws_bytes < need)) return WVAE_ERR_WORKSPACE;
+  DeviceInfo* d = nullptr;
+  wvae_status st = device_info(&d);
+  if (st != WVAE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const void* a = x;
+  if (has_norm) {
+    st = wvae_norm_silu(x, workspace, norm_gamma, norm_beta, T, H, W, cin, 1e-12f, dtype, stream);
+    if (st != WVAE_OK) return st;
+    a = workspace;
+  }
+  if (dtype == WVAE_F32) {
+    const PackedLayout L = packed_layout(cout, cin, kt, kh, kw, WVAE_F32);
+    ConvF32Params p;
+    p.x = static_cast<const float*>(a);
+    p.cache = static_cast<const float*>(cache);
+    p.w = static_cast<const float*>(packed_w);
+    p.bias = reinterpret_cast<const float*>(static_cast<const char*>(packed_w) + L.bias_off);
+    p.residual = static_cast<const float*>(residual);
+    p.y = static_cast<float*>(y);
+    p.T = T; p.H = H; p.W = W; p.cin = cin; p.cout = cout; p.KT = kt; p.KH = kh; p.KW = kw;
+    return cuda_status(launch_conv_f32(p, s));
+  }
+  TcConv c;
+  c.x = a;
+  c.cin_pad = cin;
+  c.cache = cache;
+  c.packed = packed_w;
+  c.cout = cout;
+  c.KT = kt; c.KH = kh; c.KW = kw;
+  c.T = T; c.H = H; c.W = W;
+  c.ep.residual = residual;
+  c.ep.residual_f32 = 0;
+  c.ep.out = y;
+  c.ep.out_f32 = 0;
+  return run_tc_conv(*d, c, s);
+}
+
+// ------------------------------------------------------------ residual block
+size_t wvae_resblock_workspace_bytes(int T, int H, int W, int cin, int cout, wvae_dtype dtype) {
+  if (T < 1 || H < 1 || W < 1 || cin < 1 || cout < 1) return 0;
+  const size_t nvox = static_cast<size_t>(T) * H * W;
+  const size_t c1 = dtype == WVAE_F32 ? std::max(cin, cout) : cin;
+  return round_up_sz(nvox * c1 * bytes_of(dtype), 256) + round_up_sz(nvox * cout * bytes_of(dtype), 256);
+}
+
+wvae_status wvae_resblock(const void* x, void* y, int T, int H, int W, int cin, int cout,
+                          const float* gamma1, const float* beta1, const void* w1_packed,
+                          const float* gamma2, const float* beta2, const void* w2_packed,
+                          const void* wsc_packed, wvae_dtype dtype, void* workspace,
+                          size_t ws_bytes, wvae_stream_t stream) {
+  if (!x || !y || !gamma1 || !beta1 || !w1_packed || !gamma2 || !beta2 || !w2_packed)
+    return WVAE_ERR_INVALID_ARG;
+  if (T < 1 || H < 1 || W < 1 || cin < 1 || cout < 1) return WVAE_ERR_INVALID_ARG;
+  if ((cin != cout) != (wsc_packed != nullptr)) return WVAE_ERR_INVALID_ARG;
+  if (x == y) return WVAE_ERR_INVALID_ARG;
+  if (dtype != WVAE_BF16 && dtype != WVAE_F32) return WVAE_ERR_UNSUPPORTED;
+  if (!a16(x) || !a16(y) || !a16(w1_packed) || !a16(w2_packed) || (wsc_packed && !a16(wsc_packed)) ||
+      (workspace && !a16(workspace)))
+    return WVAE_ERR_ALIGNMENT;
+  if (dtype == WVAE_BF16 && (cin % 64 != 0 || cout % 64 != 0 || !bf16_cout_ok(cout)))
+    return WVAE_ERR_UNSUPPORTED;
+  if (dtype == WVAE_F32 && (cin % 4 != 0 || cout % 4 != 0)) return WVAE_ERR_UNSUPPORTED;
+  const size_t need = wvae_resblock_workspace_bytes(T, H, W, cin, cout, dtype);
+  if (workspace == nullptr || ws_bytes < need) return WVAE_ERR_WORKSPACE;
+  DeviceInfo* d = nullptr;
+  wvae_status st = device_info(&d);
+  if (st != WVAE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t nvox = static_cast<size_t>(T) * H * W;
+  char* a1 = static_cast<char*>(workspace);
+  const size_t a1_ch = dtype == WVAE_F32 ? std::max(cin, cout) : cin;
+  char* a2 = a1 + round_up_sz(nvox * a1_ch * bytes_of(dtype), 256);
+
+  // A1 = SiLU(norm1(x))
+  st = wvae_norm_silu(x, a1, gamma1, beta1, T, H, W, cin, 1e-12f, dtype, stream);
+  if (st != WVAE_OK) return st;
+
+  if (dtype == WVAE_F32) {
+    // h1 = conv1(A1) -> a2 buffer, then A2 in place, then conv2 (+ shortcut).
+    st = wvae_causal_conv3d(a1, nullptr, w1_packed, T, H, W, cin, cout, 3, 3, 3, nullptr, nullptr,
+                            nullptr, a2, dtype, nullptr, 0, stream);
+    if (st != WVAE_OK) return st;
+    st = wvae_norm_silu(a2, a2, gamma2, beta2, T, H, W, cout, 1e-12f, dtype, stream);
+    if (st != WVAE_OK) return st;
+    const void* res = x;
+    if (wsc_packed != nullptr) {
+      // the shortcut goes to the a1 buffer (A1 is no longer needed; it is
+      // sized for max(cin, cout) channels on this path)
+      st = wvae_causal_conv3d(x, nullptr, wsc_packed, T, H, W, cin, cout, 1, 1, 1, nullptr,
+                              nullptr, nullptr, a1, dtype, nullptr, 0, stream);
+      if (st != WVAE_OK) return st;
+      res = a1;
+    }
+    return wvae_causal_conv3d(a2, nullptr, w2_packed, T, H, W, cout, cout, 3, 3, 3, nullptr,
+                              nullptr, res, y, dtype, nullptr, 0, stream);
+  }
+
+  // conv1 with norm2 + SiLU in its epilogue: writes A2 directly.
+  TcConv c1;
+  c1.x = a1;
+  c1.cin_pad = cin;
+  c1.packed = w1_packed;
+  c1.cout = cout;
+  c1.T = T; c1.H = H; c1.W = W;
+  c1.ep.act = reinterpret_cast<__nv_bfloat16*>(a2);
+  c1.ep.gamma = gamma2;
+  c1.ep.beta = beta2;
+  c1.ep.eps = 1e-12f;
+  st = run_tc_conv(*d, c1, s);
+  if (st != WVAE_OK) return st;
+
+  // conv2 (+ the 1x1x1 shortcut as a second K segment, or + x) -> y.
+  TcConv c2;
+  c2.x = a2;
+  c2.cin_pad = cout;
+  c2.packed = w2_packed;
+  c2.cout = cout;
+  c2.T = T; c2.H = H; c2.W = W;
+  if (wsc_packed != nullptr) {
+    c2.x2 = x;
+    c2.cin2_pad = cin;
+    c2.packed2 = wsc_packed;
+  } else {
+    c2.ep.residual = x;
+    c2.ep.residual_f32 = 0;
+  }
+  c2.ep.out = y;
+  c2.ep.out_f32 = 0;
+  return run_tc_conv(*d, c2, s);
+}
+
+// ------------------------------------------------------ upsample + 3x3 conv
+size_t wvae_upsample_conv_workspace_bytes(int T, int H, int W, int cin, wvae_dtype dtype) {
+  if (T < 1 || H < 1 || W < 1 || cin < 1) return 0;
+  return round_up_sz(static_cast<size_t>(T) * 4 * H * W * cin * bytes_of(dtype), 256);
+}
+
+wvae_status wvae_upsample_conv(const void* x, void* y, int T, int H, int W, int cin, int cout,
+                               const void* packed_w, wvae_dtype dtype, void* workspace,
+                               size_t ws_bytes, wvae_stream_t stream) {
+  if (!x || !y || !packed_w) return WVAE_ERR_INVALID_ARG;
+  if (T < 1 || H < 1 || W < 1 || cin < 1 || cout < 1) return WVAE_ERR_INVALID_ARG;
+  if (x == y) return WVAE_ERR_INVALID_ARG;
+  if (dtype != WVAE_BF16 && dtype != WVAE_F32) return WVAE_ERR_UNSUPPORTED;
+  if (!a16(x) || !a16(y) || !a16(packed_w) || (workspace && !a16(workspace)))
+    return WVAE_ERR_ALIGNMENT;
+  if (dtype == WVAE_BF16 && (cin % 64 != 0 || !bf16_cout_ok(cout))) return WVAE_ERR_UNSUPPORTED;
+  if (dtype == WVAE_F32 && (cin % 4 != 0 || cout % 4 != 0)) return WVAE_ERR_UNSUPPORTED;
+  const size_t need = wvae_upsample_conv_workspace_bytes(T, H, W, cin, dtype);
+  if (workspace == nullptr || ws_bytes < need) return WVAE_ERR_WORKSPACE;
+  DeviceInfo* d = nullptr;
+  wvae_status st = device_info(&d);
+  if (st != WVAE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = cuda_status(launch_upsample2x(x, workspace, static_cast<int>(bytes_of(dtype)), T, H, W, cin, s));
+  if (st != WVAE_OK) return st;
+  return wvae_causal_conv3d(workspace, nullptr, packed_w, T, 2 * H, 2 * W, cin, cout, 1, 3, 3,
+                            nullptr, nullptr, nullptr, y, dtype, nullptr, 0, stream);
+}
+
+// ------------------------------------------------------------ decoder trunk
+namespace {
+const int kDefaultWidths[4] = {512, 512, 256, 128};
+constexpr int kZChannels = 48;
+constexpr int kZPad = 64;
+constexpr int kHeadOut = 12;
+
+struct TrunkBuffers {
+  size_t zcl, h, act1, act2, up;   // byte offsets
+  size_t total;
+};
+
+TrunkBuffers trunk_buffers(int T, int H, int W, const int* C) {
+  TrunkBuffers b;
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    size_t o = off;
+    off += round_up_sz(n, 256);
+    return o;
+  };
+  const size_t v0 = static_cast<size_t>(T) * H * W;
+  size_t max_h = 0, max_act = 0, max_up = 0;
+  for (int s = 0; s < 4; ++s) {
+    const size_t vs = v0 << (2 * s);
+    max_h = std::max(max_h, vs * C[s] * 4);
+    max_act = std::max(max_act, vs * C[s] * 2);
+    if (s < 3) max_up = std::max(max_up, (vs << 2) * C[s] * 2);
+  }
+  b.zcl = take(v0 * kZPad * 2);
+  b.h = take(max_h);
+  b.act1 = take(max_act);
+  b.act2 = take(max_act);
+  b.up = take(max_up);
+  b.total = off;
+  return b;
+}
+}  // namespace
+
+size_t wvae_decode_trunk_workspace_bytes(int T, int H, int W, const int* widths) {
+  if (T < 1 || H < 1 || W < 1) return 0;
+  const int* C = widths ? widths : kDefaultWidths;
+  for (int s = 0; s < 4; ++s)
+    if (C[s] < 64) return 0;
+  return trunk_buffers(T, H, W, C).total;
+}
+
+wvae_status wvae_decode_trunk(const void* const* packed, const float* const* norms, const void* z,
+                              void* video, int T, int H, int W, const int* widths,
+                              wvae_dtype dtype, void* workspace, size_t ws_bytes,
+                              wvae_stream_t stream) {
+  if (!packed || !norms || !z || !video || !workspace) return WVAE_ERR_INVALID_ARG;
+  if (T < 1 || H < 1 || W < 1) return WVAE_ERR_INVALID_ARG;
+  if (dtype != WVAE_BF16) return WVAE_ERR_UNSUPPORTED;
+  const int* C = widths ? widths : kDefaultWidths;
+  for (int s = 0; s < 4; ++s)
+    if (C[s] % 64 != 0 || !bf16_cout_ok(C[s])) return WVAE_ERR_UNSUPPORTED;
+  for (int i = 0; i < 21; ++i)
+    if (!packed[i]) return WVAE_ERR_INVALID_ARG;
+  for (int i = 0; i < 34; ++i)
+    if (!norms[i]) return WVAE_ERR_INVALID_ARG;
+  for (int i = 0; i < 21; ++i)
+    if (!a16(packed[i])) return WVAE_ERR_ALIGNMENT;
+  if (!a16(z) || !a16(video) || !a16(workspace)) return WVAE_ERR_ALIGNMENT;
+  const TrunkBuffers B = trunk_buffers(T, H, W, C);
+  if (ws_bytes < B.total) return WVAE_ERR_WORKSPACE;
+  DeviceInfo* d = nullptr;
+  wvae_status st = device_info(&d);
+  if (st != WVAE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  void* zcl = ws + B.zcl;
+  float* h = reinterpret_cast<float*>(ws + B.h);
+  __nv_bfloat16* act[2] = {reinterpret_cast<__nv_bfloat16*>(ws + B.act1),
+                           reinterpret_cast<__nv_bfloat16*>(ws + B.act2)};
+  void* up = ws + B.up;
+
+  // latents NCDHW -> channels-last, channels padded 48 -> 64
+  st = cuda_status(launch_ncdhw_to_cl_pad(static_cast<const __nv_bfloat16*>(z),
+                                          static_cast<__nv_bfloat16*>(zcl), kZChannels, kZPad, T,
+                                          H, W, s));
+  if (st != WVAE_OK) return st;
+
+  int pi = 0, ni = 0;
+  auto next_norm = [&](const float** g, const float** b) {
+    *g = norms[2 * ni];
+    *b = norms[2 * ni + 1];
+    ++ni;
+  };
+  int Hs = H, Ws = W;
+
+  // conv_in: residual stream h (fp32) + A1 of stage 0, block 0.
+  {
+    TcConv c;
+    c.x = zcl;
+    c.cin_pad = kZPad;
+    c.packed = packed[pi++];
+    c.cout = C[0];
+    c.T = T; c.H = Hs; c.W = Ws;
+    c.ep.out = h;
+    c.ep.out_f32 = 1;
+    c.ep.act = act[0];
+    next_norm(&c.ep.gamma, &c.ep.beta);
+    c.ep.eps = 1e-12f;
+    st = run_tc_conv(*d, c, s);
+    if (st != WVAE_OK) return st;
+  }
+  for (int stg = 0; stg < 4; ++stg) {
+    const int Cs = C[stg];
+    for (int blk = 0; blk < 2; ++blk) {
+      // conv1: A1 -> A2 (norm2 in the epilogue)
+      TcConv c1;
+      c1.x = act[0];
+      c1.cin_pad = Cs;
+      c1.packed = packed[pi++];
+      c1.cout = Cs;
+      c1.T = T; c1.H = Hs; c1.W = Ws;
+      c1.ep.act = act[1];
+      next_norm(&c1.ep.gamma, &c1.ep.beta);
+      c1.ep.eps = 1e-12f;
+      st = run_tc_conv(*d, c1, s);
+      if (st != WVAE_OK) return st;
+      // conv2: h + conv2(A2) -> h (fp32, in place per voxel) and the next activation
+      TcConv c2;
+      c2.x = act[1];
+      c2.cin_pad = Cs;
+      c2.packed = packed[pi++];
+      c2.cout = Cs;
+      c2.T = T; c2.H = Hs; c2.W = Ws;
+      c2.ep.residual = h;
+      c2.ep.residual_f32 = 1;
+      const bool last_block = blk == 1;
+      if (!last_block) {
+        c2.ep.out = h;
+        c2.ep.out_f32 = 1;
+        c2.ep.act = act[0];
+        next_norm(&c2.ep.gamma, &c2.ep.beta);
+        c2.ep.eps = 1e-12f;
+      } else if (stg < 3) {
+        // the stage's output feeds only the upsample conv: write it 2x-upsampled, bf16
+        c2.ep.out = up;
+        c2.ep.out_f32 = 0;
+        c2.ep.out_upsample2x = 1;
+      } else {
+        // the last block feeds only norm_out + SiLU + head
+        c2.ep.act = act[0];
+        next_norm(&c2.ep.gamma, &c2.ep.beta);
+        c2.ep.eps = 1e-12f;
+      }
+      st = run_tc_conv(*d, c2, s);
+      if (st != WVAE_OK) return st;
+    }
+    if (stg < 3) {
+      Hs *= 2;
+      Ws *= 2;
+      TcConv cu;
+      cu.x = up;
+      cu.cin_pad = Cs;
+      cu.packed = packed[pi++];
+      cu.cout = C[stg + 1];
+      cu.KT = 1;
+      cu.T = T; cu.H = Hs; cu.W = Ws;
+      cu.ep.out = h;
+      cu.ep.out_f32 = 1;
+      cu.ep.act = act[0];
+      next_norm(&cu.ep.gamma, &cu.ep.beta);
+      cu.ep.eps = 1e-12f;
+      st = run_tc_conv(*d, cu, s);
+      if (st != WVAE_OK) return st;
+    }
+  }
+  // head: A_out -> causal conv to 12 channels -> pixel-shuffled video
+  TcConv ch;
+  ch.x = act[0];
+  ch.cin_pad = C[3];
+  ch.packed = packed[pi++];
+  ch.cout = kHeadOut;
+  ch.T = T; ch.H = Hs; ch.W = Ws;
+  ch.ep.video = static_cast<__nv_bfloat16*>(video);
+  return run_tc_conv(*d, ch, s);
+}
+
+}  // extern "C"

@@ -1,0 +1,472 @@
+// Causal conv3d as an implicit GEMM on the sm_100a tensor cores.
+//
+//   out[m, n] = sum_k A[m, k] * B[n, k]
+//   m: an output voxel (t, h, w);  n: an output channel;
+//   k: (tap, input channel), tap = (kt, kh, kw) over the KT x KH x KW window.
+//   A[m, (tap, i)] = a[t + kt - (KT-1), h + kh - (KH-1)/2, w + kw - (KW-1)/2, i]
+//
+// The causal front frames and the spatial border are zero (or, for t' < 0, the
+// previous chunk's cached frames).  No padded copy exists: every K block is one
+// TMA box load of the channels-last activation at the tap-shifted coordinates,
+// and the tensor map's out-of-bounds fill supplies the zeros.  (Conv definition:
+// FastVideo "Wan2.2 VAE decoder (sm_100a, sm_103a)" README, "Limits": bf16
+// operands, fp32 accumulation; temporal caching: TensorRT-LLM issue #19309,
+// "Feature, motivation and proposed scope".)
+//
+// One CTA per SM, persistent over output tiles of 128 voxels (8 rows x 16
+// columns of one frame) x BN output channels.  Warp roles:
+//   warp 0      TMA producer: A box {64 ch, 16 w, 8 h, 1 t} + B box {64, BN}
+//               per K block into a ring of `stages` shared-memory stages;
+//   warp 1      MMA issuer: 4 x tcgen05.mma (M=128, N=BN<=256, K=16) per K
+//               block into a TMEM accumulator (two accumulators when BN <= 256,
+//               so the epilogue of tile i overlaps the main loop of tile i+1);
+//   warps 2..5  epilogue: one TMEM lane (= one output voxel) per thread.
+// The epilogue adds bias (and residual), and may emit the raw result (fp32 or
+// bf16, optionally 2x-upsampled), the next layer's SiLU(norm(.)) activation
+// (the whole channel vector of the voxel is in the thread's TMEM lane, so the
+// RMS statistic needs no cross-thread reduction), or the 2x2 pixel-shuffled
+// NCDHW video.  An optional second K segment (the 1x1x1 shortcut of a
+// channel-changing residual block) reads its own input and weights.
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace wvae {
+
+namespace {
+
+struct Smem {
+  uint8_t* stages;        // stage s at stages + s * stage_bytes, 1024-aligned
+  uint32_t stage_bytes;
+  uint32_t a_bytes;
+  uint64_t* full;         // [kMaxStages]
+  uint64_t* empty;        // [kMaxStages]
+  uint64_t* tfull;        // [2]
+  uint64_t* tempty;       // [2]
+  uint64_t* drain;        // [1]
+  uint32_t* tmem_slot;
+  int* abort_flag;
+  float* bias;            // [512]
+  float* gamma;           // [512]
+  float* beta;            // [512]
+};
+
+constexpr uint32_t kCtrlBytes = 512 + 3 * 512 * 4;
+
+__device__ __forceinline__ Smem carve(uint8_t* raw, const ConvParams& p) {
+  Smem s;
+  uint32_t base = smem_u32(raw);
+  uint32_t pad = (1024u - (base & 1023u)) & 1023u;
+  uint8_t* al = raw + pad;
+  s.a_bytes = kBM * kBK * 2;
+  s.stage_bytes = s.a_bytes + static_cast<uint32_t>(p.BN) * kBK * 2;
+  s.stages = al;
+  uint8_t* ctrl = al + p.stages * s.stage_bytes;
+  s.full = reinterpret_cast<uint64_t*>(ctrl);
+  s.empty = s.full + kMaxStages;
+  s.tfull = s.empty + kMaxStages;
+  s.tempty = s.tfull + 2;
+  s.drain = s.tempty + 2;
+  s.tmem_slot = reinterpret_cast<uint32_t*>(s.drain + 1);
+  s.abort_flag = reinterpret_cast<int*>(s.tmem_slot + 1);
+  s.bias = reinterpret_cast<float*>(ctrl + 512);
+  s.gamma = s.bias + 512;
+  s.beta = s.gamma + 512;
+  return s;
+}
+
+struct TileCoord {
+  int n_tile, t, th, tw;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const ConvParams& p, int tile) {
+  TileCoord c;
+  c.n_tile = tile % p.n_tiles;
+  int m = tile / p.n_tiles;
+  c.tw = m % p.tiles_w;
+  m /= p.tiles_w;
+  c.th = m % p.tiles_h;
+  c.t = m / p.tiles_h;
+  return c;
+}
+
+// ------------------------------------------------------------------ producer
+__device__ void producer(const ConvParams& p, const Smem& s) {
+  const int cchunks = p.cin_pad / kBK;
+  const int kwkh = p.KH * p.KW;
+  const int b_rows = p.BN > 256 ? 256 : p.BN;
+  const int b_loads = p.BN > 256 ? 2 : 1;
+  const uint32_t b_box_bytes = static_cast<uint32_t>(b_rows) * kBK * 2;
+  uint32_t it = 0;
+  bool aborted = false;
+  for (int tile = blockIdx.x; tile < p.num_tiles && !aborted; tile += gridDim.x) {
+    const TileCoord tc = decode_tile(p, tile);
+    const int h0 = tc.th * kTileH, w0 = tc.tw * kTileW;
+    for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+      const uint32_t st = it % p.stages;
+      const uint32_t ph = (it / p.stages) & 1u;
+      if (!mbar_wait_bounded(smem_u32(&s.empty[st]), ph ^ 1u, s.abort_flag, p.err,
+                             DEVERR_TIMEOUT_PRODUCER)) {
+        aborted = true;
+        break;
+      }
+      const uint32_t bar = smem_u32(&s.full[st]);
+      const uint32_t a_dst = smem_u32(s.stages + st * s.stage_bytes);
+      const uint32_t b_dst = a_dst + s.a_bytes;
+      mbar_arrive_expect_tx(bar, s.stage_bytes);
+      if (kb < p.kblocks_main) {
+        const int tap = kb / cchunks, cc = kb - tap * cchunks;
+        const int kt = tap / kwkh, r = tap - kt * kwkh;
+        const int kh = r / p.KW, kw = r - kh * p.KW;
+        const int ts = tc.t + kt - (p.KT - 1);
+        const int hs = h0 + kh - (p.KH - 1) / 2;
+        const int ws = w0 + kw - (p.KW - 1) / 2;
+        if (ts < 0 && p.has_cache)
+          tma_load_4d(a_dst, &p.tmC, bar, cc * kBK, ws, hs, ts + p.KT - 1);
+        else
+          tma_load_4d(a_dst, &p.tmA, bar, cc * kBK, ws, hs, ts);
+        const int kcoord = tap * p.cin_pad + cc * kBK;
+        for (int l = 0; l < b_loads; ++l)
+          tma_load_2d(b_dst + l * b_box_bytes, &p.tmB, bar, kcoord, tc.n_tile * p.BN + l * 256);
+      } else {
+        const int cc = kb - p.kblocks_main;
+        tma_load_4d(a_dst, &p.tmA2, bar, cc * kBK, w0, h0, tc.t);
+        for (int l = 0; l < b_loads; ++l)
+          tma_load_2d(b_dst + l * b_box_bytes, &p.tmB2, bar, cc * kBK, tc.n_tile * p.BN + l * 256);
+      }
+    }
+  }
+  // Do not leave while copies issued by this thread may still be landing.
+  const uint32_t issued = it;
+  for (uint32_t st = 0; st < static_cast<uint32_t>(p.stages) && st < issued; ++st) {
+    const uint32_t last = st + ((issued - 1 - st) / p.stages) * p.stages;
+    const uint32_t ph = (last / p.stages) & 1u;
+    volatile int never = 0;
+    mbar_wait_bounded(smem_u32(&s.full[st]), ph, &never, p.err, DEVERR_TIMEOUT_DRAIN,
+                      kDrainLimitNs);
+  }
+}
+
+// ----------------------------------------------------------------------- MMA
+__device__ void mma_issuer(const ConvParams& p, const Smem& s, uint32_t tmem_base) {
+  const int n_inst = p.BN > 256 ? 256 : p.BN;
+  const int halves = p.BN > 256 ? 2 : 1;
+  const uint32_t idesc = umma_idesc_bf16(kBM, n_inst);
+  const uint32_t b_half_bytes = 256u * kBK * 2;
+  uint32_t it = 0, ai = 0;
+  bool aborted = false;
+  for (int tile = blockIdx.x; tile < p.num_tiles && !aborted; tile += gridDim.x, ++ai) {
+    const uint32_t acc = ai % p.num_acc;
+    const uint32_t aph = (ai / p.num_acc) & 1u;
+    if (!mbar_wait_bounded(smem_u32(&s.tempty[acc]), aph ^ 1u, s.abort_flag, p.err,
+                           DEVERR_TIMEOUT_MMA)) {
+      aborted = true;
+      break;
+    }
+    tc_fence_after();
+    const uint32_t d_tmem = tmem_base + acc * 256u;
+    for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+      const uint32_t st = it % p.stages;
+      const uint32_t ph = (it / p.stages) & 1u;
+      if (!mbar_wait_bounded(smem_u32(&s.full[st]), ph, s.abort_flag, p.err,
+                             DEVERR_TIMEOUT_MMA)) {
+        aborted = true;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t a_addr = smem_u32(s.stages + st * s.stage_bytes);
+      const uint32_t b_addr = a_addr + s.a_bytes;
+#pragma unroll
+      for (int k = 0; k < kBK / 16; ++k) {
+        const uint64_t adesc = umma_desc_sw128(a_addr + k * 32);
+        for (int hf = 0; hf < halves; ++hf) {
+          const uint64_t bdesc = umma_desc_sw128(b_addr + hf * b_half_bytes + k * 32);
+          umma_bf16(d_tmem + hf * 256u, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+        }
+      }
+      umma_commit(smem_u32(&s.empty[st]));
+    }
+    if (aborted) break;
+    umma_commit(smem_u32(&s.tfull[acc]));
+  }
+  // Every MMA issued by this thread has finished before TMEM/smem go away.
+  umma_commit(smem_u32(s.drain));
+  volatile int never = 0;
+  mbar_wait_bounded(smem_u32(s.drain), 0, &never, p.err, DEVERR_TIMEOUT_DRAIN, kDrainLimitNs);
+}
+
+// ------------------------------------------------------------------ epilogue
+template <int NC>
+__device__ __forceinline__ void tmem_load_chunk(uint32_t taddr, float (&v)[NC]);
+template <>
+__device__ __forceinline__ void tmem_load_chunk<32>(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  tmem_ld32(taddr, r);
+  tmem_wait_ld();
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+template <>
+__device__ __forceinline__ void tmem_load_chunk<16>(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  tmem_ld16(taddr, r);
+  tmem_wait_ld();
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+template <int NC>
+__device__ __forceinline__ void add_residual(const ConvEpilogue& ep, size_t off, float (&v)[NC]) {
+  if (ep.residual_f32) {
+    const float4* r = reinterpret_cast<const float4*>(static_cast<const float*>(ep.residual) + off);
+#pragma unroll
+    for (int q = 0; q < NC / 4; ++q) {
+      float4 f = r[q];
+      v[4 * q] += f.x;
+      v[4 * q + 1] += f.y;
+      v[4 * q + 2] += f.z;
+      v[4 * q + 3] += f.w;
+    }
+  } else {
+    const uint4* r =
+        reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(ep.residual) + off);
+#pragma unroll
+    for (int q = 0; q < NC / 8; ++q) {
+      uint4 u = r[q];
+      v[8 * q + 0] += bf16lo(u.x);
+      v[8 * q + 1] += bf16hi(u.x);
+      v[8 * q + 2] += bf16lo(u.y);
+      v[8 * q + 3] += bf16hi(u.y);
+      v[8 * q + 4] += bf16lo(u.z);
+      v[8 * q + 5] += bf16hi(u.z);
+      v[8 * q + 6] += bf16lo(u.w);
+      v[8 * q + 7] += bf16hi(u.w);
+    }
+  }
+}
+
+template <int NC>
+__device__ __forceinline__ void store_bf16(__nv_bfloat16* dst, const float (&v)[NC]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < NC / 8; ++q) {
+    uint4 u;
+    u.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    u.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    u.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    u.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    d[q] = u;
+  }
+}
+
+template <int NC>
+__device__ __forceinline__ void store_f32(float* dst, const float (&v)[NC]) {
+  float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int q = 0; q < NC / 4; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+// Loads columns [c0, c0 + NC) of this thread's accumulator lane and returns
+// acc + bias (+ residual) in v.
+template <int NC>
+__device__ __forceinline__ void result_chunk(const ConvParams& p, const Smem& s, uint32_t taddr,
+                                             int c0, int n0, bool valid, size_t vox,
+                                             float (&v)[NC]) {
+  tmem_load_chunk<NC>(taddr + c0, v);
+#pragma unroll
+  for (int j = 0; j < NC; ++j) v[j] += s.bias[n0 + c0 + j];
+  if (p.ep.residual != nullptr && valid)
+    add_residual<NC>(p.ep, vox * p.cout + n0 + c0, v);
+}
+
+template <int NC>
+__device__ __forceinline__ void emit_chunk(const ConvParams& p, const Smem& s, int c0, int n0,
+                                           const TileCoord& tc, int h, int w, size_t vox,
+                                           float rs, float (&v)[NC]) {
+  const ConvEpilogue& ep = p.ep;
+  if (ep.out != nullptr) {
+    if (!ep.out_upsample2x) {
+      const size_t off = vox * p.cout + n0 + c0;
+      if (ep.out_f32)
+        store_f32<NC>(static_cast<float*>(ep.out) + off, v);
+      else
+        store_bf16<NC>(static_cast<__nv_bfloat16*>(ep.out) + off, v);
+    } else {
+      const int H2 = 2 * p.H, W2 = 2 * p.W;
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const size_t v2 = (static_cast<size_t>(tc.t) * H2 + 2 * h + i) * W2 + 2 * w + j;
+          const size_t off = v2 * p.cout + n0 + c0;
+          if (ep.out_f32)
+            store_f32<NC>(static_cast<float*>(ep.out) + off, v);
+          else
+            store_bf16<NC>(static_cast<__nv_bfloat16*>(ep.out) + off, v);
+        }
+    }
+  }
+  if (ep.act != nullptr) {
+    float a[NC];
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+      const float sv = v[j] * rs * s.gamma[n0 + c0 + j] + s.beta[n0 + c0 + j];
+      a[j] = sv * __frcp_rn(1.0f + __expf(-sv));
+    }
+    store_bf16<NC>(ep.act + vox * p.cout + n0 + c0, a);
+  }
+  if (ep.video != nullptr) {
+    const int H2 = 2 * p.H, W2 = 2 * p.W;
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+      const int o = n0 + c0 + j;
+      if (o < p.cout) {
+        const int c = o >> 2, i = (o >> 1) & 1, jj = o & 1;
+        const size_t idx =
+            ((static_cast<size_t>(c) * p.T + tc.t) * H2 + 2 * h + i) * W2 + 2 * w + jj;
+        ep.video[idx] = __float2bfloat16_rn(v[j]);
+      }
+    }
+  }
+}
+
+__device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base, int warp,
+                         int lane) {
+  const int q = warp & 3;  // TMEM lane quarter this warp may access
+  const int row = q * 32 + lane;
+  const int hl = row / kTileW, wl = row % kTileW;
+  const float rootC = sqrtf(static_cast<float>(p.cout));
+  uint32_t ai = 0;
+  for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++ai) {
+    const uint32_t acc = ai % p.num_acc;
+    const uint32_t aph = (ai / p.num_acc) & 1u;
+    int ok = 0;
+    if (lane == 0)
+      ok = mbar_wait_bounded(smem_u32(&s.tfull[acc]), aph, s.abort_flag, p.err,
+                             DEVERR_TIMEOUT_EPILOGUE)
+               ? 1
+               : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) break;
+    tc_fence_after();
+    const TileCoord tc = decode_tile(p, tile);
+    const int h = tc.th * kTileH + hl, w = tc.tw * kTileW + wl;
+    const bool valid = h < p.H && w < p.W;
+    const size_t vox = (static_cast<size_t>(tc.t) * p.H + h) * p.W + w;
+    const int n0 = tc.n_tile * p.BN;
+    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * 256u;
+
+    float rs = 1.0f;
+    if (p.ep.act != nullptr) {
+      float ss = 0.0f;
+      int c0 = 0;
+      for (; c0 + 32 <= p.BN; c0 += 32) {
+        float v[32];
+        result_chunk<32>(p, s, taddr, c0, n0, valid, vox, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
+      }
+      if (c0 < p.BN) {
+        float v[16];
+        result_chunk<16>(p, s, taddr, c0, n0, valid, vox, v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) ss = fmaf(v[j], v[j], ss);
+      }
+      rs = rootC / fmaxf(sqrtf(ss), p.ep.eps);
+    }
+    int c0 = 0;
+    for (; c0 + 32 <= p.BN; c0 += 32) {
+      float v[32];
+      result_chunk<32>(p, s, taddr, c0, n0, valid, vox, v);
+      if (valid) emit_chunk<32>(p, s, c0, n0, tc, h, w, vox, rs, v);
+    }
+    if (c0 < p.BN) {
+      float v[16];
+      result_chunk<16>(p, s, taddr, c0, n0, valid, vox, v);
+      if (valid) emit_chunk<16>(p, s, c0, n0, tc, h, w, vox, rs, v);
+    }
+    tc_fence_before();
+    mbar_arrive(smem_u32(&s.tempty[acc]));
+  }
+}
+
+__global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_constant__ ConvParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const Smem s = carve(smem_raw, p);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < p.stages; ++i) {
+      mbar_init(smem_u32(&s.full[i]), 1);
+      mbar_init(smem_u32(&s.empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&s.tfull[i]), 1);
+      mbar_init(smem_u32(&s.tempty[i]), 128);
+    }
+    mbar_init(smem_u32(s.drain), 1);
+    *s.abort_flag = 0;
+    fence_mbar_init();
+  }
+  // Per-channel vectors for every output channel (a CTA may visit several
+  // n-slices); the shortcut bias folds into the bias.
+  for (int i = threadIdx.x; i < p.cout_pad; i += blockDim.x) {
+    s.bias[i] = p.ep.bias[i] + (p.ep.bias2 != nullptr ? p.ep.bias2[i] : 0.0f);
+    if (p.ep.act != nullptr && i < p.cout) {
+      s.gamma[i] = p.ep.gamma[i];
+      s.beta[i] = p.ep.beta[i];
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(s.tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tmA);
+    tma_prefetch_desc(&p.tmB);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s.tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) producer(p, s);
+  } else if (warp == 1) {
+    if (lane == 0) mma_issuer(p, s, tmem_base);
+  } else {
+    epilogue(p, s, tmem_base, warp, lane);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace
+
+size_t conv_tc_smem_bytes(int BN, int stages) {
+  const size_t stage = static_cast<size_t>(kBM) * kBK * 2 + static_cast<size_t>(BN) * kBK * 2;
+  return 1024 + stages * stage + kCtrlBytes;
+}
+
+int conv_tc_stages_for(int BN) {
+  const size_t limit = 232448;  // 227 KB opt-in dynamic shared memory per block
+  int st = kMaxStages;
+  while (st > 2 && conv_tc_smem_bytes(BN, st) > limit) --st;
+  return st;
+}
+
+cudaError_t launch_conv_tc(const ConvParams& p, int grid, cudaStream_t stream) {
+  const size_t smem = conv_tc_smem_bytes(p.BN, p.stages);
+  cudaError_t e = cudaFuncSetAttribute(conv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  conv_tc_kernel<<<grid, kConvThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace wvae

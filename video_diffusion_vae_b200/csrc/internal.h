@@ -1,0 +1,98 @@
+// Host/device shared declarations of the library's internal launch interface.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace wvae {
+
+// ----------------------------------------------------------- conv (tcgen05)
+// Output tile: 128 voxels of one frame, 8 rows x 16 columns; K block: 64
+// input channels of one tap.
+constexpr int kTileH = 8;
+constexpr int kTileW = 16;
+constexpr int kBM = kTileH * kTileW;  // 128
+constexpr int kBK = 64;
+constexpr int kConvThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kMaxStages = 8;
+
+// What the epilogue does with acc + bias (+ residual), per output voxel.
+struct ConvEpilogue {
+  const float* bias;        // fp32 [cout_pad] (packed blob)
+  const float* bias2;       // fp32 [cout_pad] shortcut bias, or null
+  const void* residual;     // [T][H][W][cout] or null
+  int residual_f32;         // residual dtype: 1 fp32, 0 bf16
+  void* out;                // raw result [T][H][W][cout] (or [T][2H][2W][cout]), or null
+  int out_f32;              // out dtype: 1 fp32, 0 bf16
+  int out_upsample2x;       // 1: write each voxel to its 2x2 block at double resolution
+  __nv_bfloat16* act;       // SiLU(norm(result)) bf16 [T][H][W][cout], or null
+  const float* gamma;       // fp32 [cout] for act
+  const float* beta;        // fp32 [cout] for act
+  float eps;
+  __nv_bfloat16* video;     // 2x2 pixel-shuffled NCDHW [cout/4][T][2H][2W], or null
+};
+
+struct ConvParams {
+  CUtensorMap tmA;   // main input, bf16 [T][H][W][cin_pad], box {64, 16, 8, 1}
+  CUtensorMap tmB;   // main weights, bf16 [cout_pad][taps * cin_pad], box {64, <=256}
+  CUtensorMap tmC;   // cached frames, bf16 [KT-1][H][W][cin_pad] (has_cache)
+  CUtensorMap tmA2;  // shortcut input, bf16 [T][H][W][cin2_pad] (cin2_pad > 0)
+  CUtensorMap tmB2;  // shortcut weights, bf16 [cout_pad][cin2_pad]
+  int T, H, W;
+  int cin_pad, cin2_pad;
+  int cout, cout_pad;
+  int KT, KH, KW;
+  int has_cache;
+  int BN, n_tiles;
+  int tiles_w, tiles_h, m_tiles, num_tiles;
+  int stages, num_acc;
+  int kblocks_main, kblocks;
+  ConvEpilogue ep;
+  unsigned* err;
+};
+
+size_t conv_tc_smem_bytes(int BN, int stages);
+int conv_tc_stages_for(int BN);
+cudaError_t launch_conv_tc(const ConvParams& p, int grid, cudaStream_t stream);
+
+// ------------------------------------------------------------ fp32 direct conv
+struct ConvF32Params {
+  const float* x;      // [T][H][W][cin]
+  const float* cache;  // [KT-1][H][W][cin] or null
+  const float* w;      // packed fp32 [taps][cin][cout]
+  const float* bias;   // [cout]
+  const float* residual;
+  float* y;            // [T][H][W][cout]
+  int T, H, W, cin, cout, KT, KH, KW;
+};
+cudaError_t launch_conv_f32(const ConvF32Params& p, cudaStream_t stream);
+
+// ---------------------------------------------------------------- norm-SiLU
+cudaError_t launch_norm_silu_bf16(const __nv_bfloat16* x, __nv_bfloat16* y, const float* gamma,
+                                  const float* beta, long nvox, int C, float eps, int num_sms,
+                                  cudaStream_t stream);
+cudaError_t launch_norm_silu_f32(const float* x, float* y, const float* gamma, const float* beta,
+                                 long nvox, int C, float eps, int num_sms, cudaStream_t stream);
+
+// ------------------------------------------------------------ layout kernels
+cudaError_t launch_prepack_bf16(const void* w, int w_is_f32, const float* bias, int cout, int cin,
+                                int taps, int cout_pad, int cin_pad, __nv_bfloat16* wp,
+                                float* bias_p, cudaStream_t stream);
+cudaError_t launch_prepack_f32(const void* w, int w_is_f32, const float* bias, int cout, int cin,
+                               int taps, float* wp, float* bias_p, cudaStream_t stream);
+// NCDHW [C][T][H][W] bf16 -> channels-last [T][H][W][Cpad] bf16, zero-filled pad channels.
+cudaError_t launch_ncdhw_to_cl_pad(const __nv_bfloat16* x, __nv_bfloat16* y, int C, int Cpad,
+                                   int T, int H, int W, cudaStream_t stream);
+// channels-last [T][H][W][C] -> [T][2H][2W][C], nearest.
+cudaError_t launch_upsample2x(const void* x, void* y, int elem_bytes, int T, int H, int W, int C,
+                              cudaStream_t stream);
+// fp32 [n] -> bf16 [n]
+cudaError_t launch_f32_to_bf16(const float* x, __nv_bfloat16* y, size_t n, cudaStream_t stream);
+
+// Device error word (defined in api.cu).
+unsigned* device_error_word();
+
+}  // namespace wvae
