@@ -1,0 +1,442 @@
+"""Benchmark of the Wan-style video-VAE decoder hot path on B200.
+
+One step = one decode of the Wan2.2-shaped decoder trunk (latents
+[1, 48, 4, 44, 78] -> video [1, 3, 4, 704, 1248], bf16, random weights with the
+trunk's shapes): conv_in, 8 residual blocks (norm + SiLU fused into the conv
+epilogues, causal 3x3x3 convs, residual adds), 3 nearest-2x upsample convs and
+norm_out + SiLU + head conv + pixel shuffle.  It runs every step of the hot
+path; value = decoded frames/s over all ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank decodes its own replica (the trunk has no exchange
+step: "replicas only"); the timed region is bracketed by a barrier and a
+device synchronise and its duration is the max over ranks.  `--impl
+reference` times the CPU oracle instead (rank 0 only), on a bounded sample.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "res-block conv TFLOP/s (% bf16 peak); norm-SiLU GB/s (% HBM); frames/s"
+UNIT = "frames/s"
+T, H, W = 4, 44, 78
+WIDTHS = (512, 512, 256, 128)
+ZC = 48
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 512 << 20
+
+
+# ------------------------------------------------------------------ workload
+def trunk_layers(T=T, H=H, W=W, widths=WIDTHS, zc=ZC):
+    """The trunk's launches in order with their dense FLOPs (all taps counted)."""
+    layers = [("layout", 0.0)]
+    v = T * H * W
+    layers.append(("conv_in", 2.0 * v * widths[0] * zc * 27))
+    for s, c in enumerate(widths):
+        vs = v * 4 ** s
+        for b in range(2):
+            layers.append((f"s{s}.b{b}.conv1", 2.0 * vs * c * c * 27))
+            layers.append((f"s{s}.b{b}.conv2", 2.0 * vs * c * c * 27))
+        if s + 1 < len(widths):
+            layers.append((f"s{s}.up", 2.0 * (4 * vs) * widths[s + 1] * c * 9))
+    v3 = v * 4 ** (len(widths) - 1)
+    layers.append(("head", 2.0 * v3 * 12 * widths[-1] * 27))
+    return layers
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) >= 9:
+                    rows.append(f)
+        except Exception:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------- CPU baseline
+def oracle_trunk_sample(h=4, w=6):
+    """Time the CPU oracle on the trunk at latents [1, 48, 4, h, w] (full channel
+    widths) and scale to the full 44 x 78 workload by the dense FLOP ratio."""
+    from oracle import oracle as O
+    from video_diffusion_vae_b200 import synth
+    z, params = synth.trunk_input(T=T, H=h, W=w, seed=1)
+    t0 = time.perf_counter()
+    O.trunk(z, params)
+    dt = time.perf_counter() - t0
+    f_sample = sum(f for _, f in trunk_layers(T, h, w))
+    f_full = sum(f for _, f in trunk_layers())
+    fps = T / (dt * f_full / f_sample)
+    return fps, dt, O.nthreads(), f"oracle trunk on latents [1,48,{T},{h},{w}] (full widths), " \
+        f"{dt:.1f} s, scaled by dense FLOPs {f_full / f_sample:.0f}x to [1,48,{T},{H},{W}]"
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    vals = []
+    for i in range(args.warmup + args.steps):
+        fps, dt, cores, sample = oracle_trunk_sample(2, 3)
+        if i >= args.warmup:
+            vals.append(fps)
+    v = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": T / v * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "Wan2.2-shaped decoder trunk, latents [1,48,4,44,78] -> video "
+                               "[1,3,4,704,1248], widths 512/512/256/128, 2 res blocks per stage",
+                   "sample": sample},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# -------------------------------------------------------------- components
+def time_events(fn, reps, warm, flush):
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn()
+        e.record()
+        e.synchronize()
+        ts.append(s.elapsed_time(e))
+    return statistics.median(ts), min(ts)
+
+
+def components(peaks, flush, reps=10):
+    """Per-kernel figures of the metric on their own workloads: norm-SiLU GB/s on
+    [512,4,88,156] / [256,4,176,312], the causal conv 512->512 on [512,4,88,156],
+    and the res block 256->256 (and 256->128) on [256,4,176,312]."""
+    import torch
+    from video_diffusion_vae_b200 import binding as B
+    from video_diffusion_vae_b200 import synth
+    out = {}
+    for shp in [(512, 4, 88, 156), (256, 4, 176, 312)]:
+        x, g, b = synth.norm_silu_input(*shp)
+        xd = x.permute(1, 2, 3, 0).contiguous().cuda().bfloat16()
+        gd, bd = g.cuda(), b.cuda()
+        y = torch.empty_like(xd)
+        med, mn = time_events(lambda: B.norm_silu(xd, gd, bd, out=y), reps, 3, flush)
+        gbs = 2 * xd.numel() * 2 / (med * 1e-3) / 1e9
+        out[f"norm_silu_{'x'.join(map(str, shp))}"] = {
+            "ms": med, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"], "frac_8TBs": gbs / 8000.0}
+        del xd, y
+    x, w, b = synth.conv_input()
+    pk = B.prepack_conv(w.cuda().bfloat16(), b.cuda())
+    xd = x.permute(1, 2, 3, 0).contiguous().cuda().bfloat16()
+    y = torch.empty_like(xd)
+    med, mn = time_events(lambda: B.causal_conv3d(xd, pk, out=y), reps, 3, flush)
+    fl = 2.0 * 512 * 512 * 27 * 4 * 88 * 156
+    out["conv_512x512_4x88x156"] = {"ms": med, "TFLOP/s": fl / med / 1e9,
+                                    "frac_bf16": fl / med / 1e9 / peaks["bf16_tflops"],
+                                    "frac_2250": fl / med / 1e9 / 2250.0}
+    del xd, y, pk
+    for cout in (256, 128):
+        x, p = synth.resblock_input(cout=cout)
+        blk = B.PackedResBlock(p)
+        xd = x.permute(1, 2, 3, 0).contiguous().cuda().bfloat16()
+        y = torch.empty((4, 176, 312, cout), dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(B.load().wvae_resblock_workspace_bytes(4, 176, 312, 256, cout, 0),
+                         dtype=torch.uint8, device="cuda")
+        med, mn = time_events(lambda: B.resblock(xd, blk, out=y, workspace=ws), reps, 3, flush)
+        nv = 4 * 176 * 312
+        fl = 2.0 * nv * 27 * (256 * cout + cout * cout) + (2.0 * nv * 256 * cout if cout != 256 else 0)
+        out[f"resblock_256x{cout}_4x176x312"] = {"ms": med, "TFLOP/s": fl / med / 1e9,
+                                                 "frac_bf16": fl / med / 1e9 / peaks["bf16_tflops"],
+                                                 "frac_2250": fl / med / 1e9 / 2250.0}
+        del xd, y, ws, blk
+    return out
+
+
+# ----------------------------------------------------- multi-rank timing
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank number over all ranks (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(frames_per_step: int, steps: int, world: int, max_total_ms: float) -> float:
+    """Whole-job frames/s: every rank decodes `steps` steps; time = slowest rank."""
+    return frames_per_step * steps * world / (max_total_ms * 1e-3)
+
+
+# ------------------------------------------------------------ profile cases
+def profile_case(name: str, launches: int = 3) -> int:
+    """Run one kernel workload `launches` times (for an ncu capture; no JSON line).
+    conv512: causal conv 512->512 on [4,88,156]; norm512 / norm256: norm-SiLU on
+    [512,4,88,156] / [256,4,176,312]; res256: res block 256->256 on [4,176,312];
+    trunk: one trunk decode."""
+    import torch
+    from video_diffusion_vae_b200 import binding as B
+    from video_diffusion_vae_b200 import synth
+    torch.cuda.set_device(0)
+    if name == "conv512":
+        x, w, b = synth.conv_input()
+        pk = B.prepack_conv(w.cuda().bfloat16(), b.cuda())
+        xd = x.permute(1, 2, 3, 0).contiguous().cuda().bfloat16()
+        fn = lambda: B.causal_conv3d(xd, pk)  # noqa: E731
+    elif name in ("norm512", "norm256"):
+        shp = (512, 4, 88, 156) if name == "norm512" else (256, 4, 176, 312)
+        x, g, b = synth.norm_silu_input(*shp)
+        xd = x.permute(1, 2, 3, 0).contiguous().cuda().bfloat16()
+        gd, bd = g.cuda(), b.cuda()
+        fn = lambda: B.norm_silu(xd, gd, bd)  # noqa: E731
+    elif name == "res256":
+        x, p = synth.resblock_input()
+        blk = B.PackedResBlock(p)
+        xd = x.permute(1, 2, 3, 0).contiguous().cuda().bfloat16()
+        fn = lambda: B.resblock(xd, blk)  # noqa: E731
+    elif name == "trunk":
+        z, params = synth.trunk_input()
+        tr = B.PackedTrunk(params)
+        zd = z[None].cuda().bfloat16().contiguous()
+        fn = lambda: B.decode_trunk(zd, tr)  # noqa: E731
+    else:
+        raise SystemExit(f"unknown profile case {name}")
+    for _ in range(launches):
+        fn()
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    return 0
+
+
+# ------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-components", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", default=None,
+                    help="run one kernel workload for an ncu capture (conv512, norm512, norm256, "
+                         "res256, trunk) and exit")
+    args = ap.parse_args()
+    if args.profile_case:
+        return profile_case(args.profile_case)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    args.warmup = max(args.warmup, 3)
+
+    import torch
+    import torch.distributed as dist
+    from video_diffusion_vae_b200 import binding as B
+    from video_diffusion_vae_b200 import synth
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+    peaks, peak_kind = load_peaks()
+
+    z, params = synth.trunk_input(T=T, H=H, W=W, seed=0)
+    tr = B.PackedTrunk(params, device=dev)
+    zd = z[None].to(dev, torch.bfloat16).contiguous()
+    video = torch.empty((1, 3, T, 16 * H, 16 * W), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(tr.workspace_bytes(T, H, W), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    layers = trunk_layers()
+    nl = B.trunk_launches()
+    assert nl == len(layers)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nl)] for _ in range(args.steps)]
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+
+    def step():
+        B.decode_trunk(zd, tr, out=video, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, L2 flushed before each (outside the step events)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()
+            step_ev[i][0].record()
+            B.decode_trunk(zd, tr, out=video, workspace=ws, events=ev[i])
+            step_ev[i][1].record()
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t0
+    if world > 1:
+        dist.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    total_ms = sum(step_ms)
+    max_total_ms = max_over_ranks(total_ms, dev)
+    value = throughput(T, args.steps, world, max_total_ms)
+    clocks = clk.summary()
+
+    # per-launch durations -> the dominant kernel (tensor-core conv) and shares
+    per_layer = [[ev[i][2 * j].elapsed_time(ev[i][2 * j + 1]) for j in range(nl)] for i in range(args.steps)]
+    conv_idx = [j for j, (name, _) in enumerate(layers) if name != "layout"]
+    conv_ms = statistics.mean(sum(per_layer[i][j] for j in conv_idx) for i in range(args.steps))
+    conv_flops = sum(layers[j][1] for j in conv_idx)
+    conv_launch_ms = conv_ms / len(conv_idx)
+    achieved = conv_flops / len(conv_idx) / (conv_launch_ms * 1e-3) / 1e12
+    layer_ms = {layers[j][0]: statistics.mean(per_layer[i][j] for i in range(args.steps)) for j in range(nl)}
+
+    # ---- e2e: pinned host latents -> device, decode, video -> pinned host, per step
+    zh = z[None].to(torch.bfloat16).contiguous().pin_memory()
+    vh = torch.empty(video.shape, dtype=torch.bfloat16).pin_memory()
+    for _ in range(2):
+        zd.copy_(zh, non_blocking=True)
+        step()
+        vh.copy_(video, non_blocking=True)
+    torch.cuda.synchronize()
+    e2e_ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        zd.copy_(zh, non_blocking=True)
+        step()
+        vh.copy_(video, non_blocking=True)
+        e.record()
+        e.synchronize()
+        e2e_ms.append(s.elapsed_time(e))
+    e2e_value = throughput(T, args.steps, world, max_over_ranks(sum(e2e_ms), dev))
+
+    err = B.device_error()
+    comp = None
+    if rank == 0 and not args.no_components:
+        del ws
+        comp = components(peaks, flush)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        fps, dt, cores, sample = oracle_trunk_sample()
+        cpu = {"value": fps, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        peak_t = peaks["bf16_tflops_sustained"]
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": max_total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) latents, random weights with the trunk's shapes)",
+            "config": {"workload": "Wan2.2-shaped decoder trunk: latents [1,48,4,44,78] -> video "
+                                   "[1,3,4,704,1248]; conv_in, 4 stages of 2 res blocks (widths "
+                                   "512/512/256/128), 3 nearest-2x upsample convs, norm_out+SiLU+head "
+                                   "conv + 2x2 pixel shuffle",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "flushed (512 MiB write) before every timed step, outside the step events",
+                       "trunk_dense_tflop_per_step": sum(f for _, f in layers) / 1e12},
+            "tflops": sum(f for _, f in layers) * args.steps / (total_ms * 1e-3) / 1e12,
+            "roofline": {"bound": "tensor", "kernel": "conv_tc_kernel (all 21 conv launches of a step)",
+                         "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
+                         "frac": achieved / peak_t, "peak_kind": f"{peak_kind} bf16 sustained",
+                         "frac_of_burst": achieved / peaks["bf16_tflops"], "frac_of_2250": achieved / 2250.0,
+                         "traffic": None, "launch_ms": conv_launch_ms,
+                         "conv_share_of_step": conv_ms / statistics.mean(step_ms)},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": zh.numel() * 2,
+                    "d2h_bytes_per_step": vh.numel() * 2},
+            "gpu_launches": nl * args.steps,
+            "clocks": clocks,
+            "wall_s_timed_region": wall,
+            "layer_ms": layer_ms,
+            "components": comp,
+            "device_error_word": err,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -189,6 +189,24 @@ WVAE_API wvae_status wvae_decode_trunk(const void* const* packed, const float* c
                               wvae_dtype dtype, void* workspace, size_t ws_bytes,
                               wvae_stream_t stream);
 
+/*
+ * Per-launch timing of the trunk.  wvae_decode_trunk enqueues exactly
+ * wvae_decode_trunk_launches() kernels on `stream`, in this order:
+ *   [0] latents NCDHW -> channels-last, [1] conv_in, then per stage s = 0..3:
+ *   block 0 conv1, block 0 conv2, block 1 conv1, block 1 conv2 and, for s < 3,
+ *   the upsample conv; the last launch is the head.
+ * wvae_decode_trunk_timed does the same work and records events[2i] just
+ * before and events[2i+1] just after launch i on `stream`.  events: host array
+ * of n_events >= 2 * launches cudaEvent_t handles created by the caller
+ * (with timing enabled); the library only records them.
+ */
+WVAE_API int wvae_decode_trunk_launches(void);
+WVAE_API wvae_status wvae_decode_trunk_timed(const void* const* packed, const float* const* norms,
+                                    const void* z, void* video, int T, int H, int W,
+                                    const int* widths, wvae_dtype dtype, void* workspace,
+                                    size_t ws_bytes, void* const* events, int n_events,
+                                    wvae_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -20,7 +20,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     declared = B.header_symbols()
-    assert len(declared) == 14
+    assert len(declared) == 16
     out = subprocess.check_output(["nm", "-D", "--defined-only", B.LIB_PATH], text=True)
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
     missing = [s for s in declared if s not in exported]
@@ -122,6 +122,12 @@ def test_trunk_rejects_on_host(lib):
     P0 = (ctypes.c_void_p * 21)(*([0x10000] * 20 + [0]))
     assert f(P0, N, A, y, 4, 44, 78, None, B.BF16, A, 1 << 40, s) == 1
     assert f(P, N, A, y, 4, 44, 78, None, B.BF16, A, 1 << 40, s) == 7
+    assert lib.wvae_decode_trunk_launches() == 22
+    E = (ctypes.c_void_p * 44)(*([0x30000] * 44))
+    ft = lib.wvae_decode_trunk_timed
+    assert ft(P, N, A, y, 4, 44, 78, None, B.BF16, A, 1 << 40, None, 0, s) == 1
+    assert ft(P, N, A, y, 4, 44, 78, None, B.BF16, A, 1 << 40, E, 43, s) == 1
+    assert ft(P, N, A, y, 4, 44, 78, None, B.BF16, A, 1 << 40, E, 44, s) == 7
 
 
 def test_binding_fails_loudly_without_library(tmp_path):

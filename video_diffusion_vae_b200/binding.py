@@ -65,6 +65,9 @@ def load(path: str | None = None):
             "wvae_decode_trunk_workspace_bytes": (S, [I, I, I, ctypes.POINTER(I)]),
             "wvae_decode_trunk": (I, [ctypes.POINTER(V), ctypes.POINTER(V), V, V, I, I, I,
                                       ctypes.POINTER(I), I, V, S, V]),
+            "wvae_decode_trunk_launches": (I, []),
+            "wvae_decode_trunk_timed": (I, [ctypes.POINTER(V), ctypes.POINTER(V), V, V, I, I, I,
+                                            ctypes.POINTER(I), I, V, S, ctypes.POINTER(V), I, V]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -282,8 +285,15 @@ class PackedTrunk:
         return load().wvae_decode_trunk_workspace_bytes(T, H, W, self._widths_arr)
 
 
-def decode_trunk(z, trunk: PackedTrunk, out=None, workspace=None):
-    """z: latents [1, 48, T, H, W] bf16 (CUDA) -> video [1, 3, T, 16H, 16W] bf16."""
+def trunk_launches() -> int:
+    return load().wvae_decode_trunk_launches()
+
+
+def decode_trunk(z, trunk: PackedTrunk, out=None, workspace=None, events=None):
+    """z: latents [1, 48, T, H, W] bf16 (CUDA) -> video [1, 3, T, 16H, 16W] bf16.
+
+    events: optional list of 2 * trunk_launches() torch.cuda.Event(enable_timing=True);
+    events[2i] / events[2i+1] are recorded around the trunk's i-th kernel launch."""
     _cuda(z, "z", torch.bfloat16)
     _, zc, T, H, W = z.shape
     if zc != 48 or z.shape[0] != 1:
@@ -292,7 +302,18 @@ def decode_trunk(z, trunk: PackedTrunk, out=None, workspace=None):
         else _cuda(out, "out", torch.bfloat16, (1, 3, T, 16 * H, 16 * W))
     nws = trunk.workspace_bytes(T, H, W)
     ws = _workspace(nws, z.device) if workspace is None else workspace
-    _check("wvae_decode_trunk", load().wvae_decode_trunk(
+    if events is None:
+        _check("wvae_decode_trunk", load().wvae_decode_trunk(
+            trunk._packed_arr, trunk._norm_arr, _ptr(z), _ptr(y), T, H, W, trunk._widths_arr, BF16,
+            _ptr(ws), ws.numel(), _stream()))
+        return y
+    handles = []
+    for ev in events:
+        if not ev.cuda_event:
+            ev.record()          # creates the underlying cudaEvent_t
+        handles.append(ev.cuda_event)
+    arr = (ctypes.c_void_p * len(handles))(*handles)
+    _check("wvae_decode_trunk_timed", load().wvae_decode_trunk_timed(
         trunk._packed_arr, trunk._norm_arr, _ptr(z), _ptr(y), T, H, W, trunk._widths_arr, BF16,
-        _ptr(ws), ws.numel(), _stream()))
+        _ptr(ws), ws.numel(), arr, len(handles), _stream()))
     return y

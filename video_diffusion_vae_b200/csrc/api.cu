@@ -539,11 +539,15 @@ size_t wvae_decode_trunk_workspace_bytes(int T, int H, int W, const int* widths)
   return trunk_buffers(T, H, W, C).total;
 }
 
-wvae_status wvae_decode_trunk(const void* const* packed, const float* const* norms, const void* z,
+namespace {
+constexpr int kTrunkLaunches = 22;
+
+wvae_status decode_trunk_impl(const void* const* packed, const float* const* norms, const void* z,
                               void* video, int T, int H, int W, const int* widths,
                               wvae_dtype dtype, void* workspace, size_t ws_bytes,
-                              wvae_stream_t stream) {
+                              void* const* events, int n_events, wvae_stream_t stream) {
   if (!packed || !norms || !z || !video || !workspace) return WVAE_ERR_INVALID_ARG;
+  if (events != nullptr && n_events < 2 * kTrunkLaunches) return WVAE_ERR_INVALID_ARG;
   if (T < 1 || H < 1 || W < 1) return WVAE_ERR_INVALID_ARG;
   if (dtype != WVAE_BF16) return WVAE_ERR_UNSUPPORTED;
   const int* C = widths ? widths : kDefaultWidths;
@@ -562,6 +566,18 @@ wvae_status wvae_decode_trunk(const void* const* packed, const float* const* nor
   wvae_status st = device_info(&d);
   if (st != WVAE_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int launch = 0;
+  auto mark = [&](int which) {
+    if (events != nullptr)
+      cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[2 * launch + which]), s);
+  };
+  auto conv = [&](const TcConv& c) {
+    mark(0);
+    wvae_status r = run_tc_conv(*d, c, s);
+    mark(1);
+    ++launch;
+    return r;
+  };
   char* ws = static_cast<char*>(workspace);
   void* zcl = ws + B.zcl;
   float* h = reinterpret_cast<float*>(ws + B.h);
@@ -570,9 +586,12 @@ wvae_status wvae_decode_trunk(const void* const* packed, const float* const* nor
   void* up = ws + B.up;
 
   // latents NCDHW -> channels-last, channels padded 48 -> 64
+  mark(0);
   st = cuda_status(launch_ncdhw_to_cl_pad(static_cast<const __nv_bfloat16*>(z),
                                           static_cast<__nv_bfloat16*>(zcl), kZChannels, kZPad, T,
                                           H, W, s));
+  mark(1);
+  ++launch;
   if (st != WVAE_OK) return st;
 
   int pi = 0, ni = 0;
@@ -596,7 +615,7 @@ wvae_status wvae_decode_trunk(const void* const* packed, const float* const* nor
     c.ep.act = act[0];
     next_norm(&c.ep.gamma, &c.ep.beta);
     c.ep.eps = 1e-12f;
-    st = run_tc_conv(*d, c, s);
+    st = conv(c);
     if (st != WVAE_OK) return st;
   }
   for (int stg = 0; stg < 4; ++stg) {
@@ -612,7 +631,7 @@ wvae_status wvae_decode_trunk(const void* const* packed, const float* const* nor
       c1.ep.act = act[1];
       next_norm(&c1.ep.gamma, &c1.ep.beta);
       c1.ep.eps = 1e-12f;
-      st = run_tc_conv(*d, c1, s);
+      st = conv(c1);
       if (st != WVAE_OK) return st;
       // conv2: h + conv2(A2) -> h (fp32, in place per voxel) and the next activation
       TcConv c2;
@@ -641,7 +660,7 @@ wvae_status wvae_decode_trunk(const void* const* packed, const float* const* nor
         next_norm(&c2.ep.gamma, &c2.ep.beta);
         c2.ep.eps = 1e-12f;
       }
-      st = run_tc_conv(*d, c2, s);
+      st = conv(c2);
       if (st != WVAE_OK) return st;
     }
     if (stg < 3) {
@@ -659,7 +678,7 @@ wvae_status wvae_decode_trunk(const void* const* packed, const float* const* nor
       cu.ep.act = act[0];
       next_norm(&cu.ep.gamma, &cu.ep.beta);
       cu.ep.eps = 1e-12f;
-      st = run_tc_conv(*d, cu, s);
+      st = conv(cu);
       if (st != WVAE_OK) return st;
     }
   }
@@ -671,7 +690,28 @@ wvae_status wvae_decode_trunk(const void* const* packed, const float* const* nor
   ch.cout = kHeadOut;
   ch.T = T; ch.H = Hs; ch.W = Ws;
   ch.ep.video = static_cast<__nv_bfloat16*>(video);
-  return run_tc_conv(*d, ch, s);
+  return conv(ch);
+}
+}  // namespace
+
+int wvae_decode_trunk_launches(void) { return kTrunkLaunches; }
+
+wvae_status wvae_decode_trunk(const void* const* packed, const float* const* norms, const void* z,
+                              void* video, int T, int H, int W, const int* widths,
+                              wvae_dtype dtype, void* workspace, size_t ws_bytes,
+                              wvae_stream_t stream) {
+  return decode_trunk_impl(packed, norms, z, video, T, H, W, widths, dtype, workspace, ws_bytes,
+                           nullptr, 0, stream);
+}
+
+wvae_status wvae_decode_trunk_timed(const void* const* packed, const float* const* norms,
+                                    const void* z, void* video, int T, int H, int W,
+                                    const int* widths, wvae_dtype dtype, void* workspace,
+                                    size_t ws_bytes, void* const* events, int n_events,
+                                    wvae_stream_t stream) {
+  if (events == nullptr) return WVAE_ERR_INVALID_ARG;
+  return decode_trunk_impl(packed, norms, z, video, T, H, W, widths, dtype, workspace, ws_bytes,
+                           events, n_events, stream);
 }
 
 }  // extern "C"

@@ -11,9 +11,10 @@
 // HBM-bound: one read and one write of the tensor.  A group of L lanes owns a
 // voxel (L = 32 for C >= 256); each lane moves 16-byte vectors (8 bf16 / 4 fp32
 // channels), so a warp's accesses to a voxel are one contiguous, fully
-// coalesced run.  The sum of squares is reduced with shuffles inside the
-// group.  Each lane keeps its channels' gamma/beta in registers for the whole
-// grid-stride loop; two voxel groups are in flight per iteration.
+// coalesced run.  Each warp first issues the loads of U voxel groups (kept
+// packed in registers), then reduces the sums of squares with shuffles inside
+// each group and writes the results; gamma/beta sit in shared memory.  The grid
+// is persistent: exactly the blocks that fit on the GPU at once.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -26,82 +27,85 @@ constexpr int kNormThreads = 256;
 __device__ __forceinline__ float silu_fast(float s) { return s * __frcp_rn(1.0f + __expf(-s)); }
 __device__ __forceinline__ float silu_exact(float s) { return s / (1.0f + expf(-s)); }
 
-// VEC = channels per 16-byte vector (8 for bf16, 4 for fp32); CH = vectors per lane.
-template <typename T, int VEC, int CH, int UNROLL>
+template <int VEC>
+__device__ __forceinline__ void unpack(const uint4& r, float (&v)[VEC]) {
+  if constexpr (VEC == 8) {
+    v[0] = bf16lo(r.x); v[1] = bf16hi(r.x); v[2] = bf16lo(r.y); v[3] = bf16hi(r.y);
+    v[4] = bf16lo(r.z); v[5] = bf16hi(r.z); v[6] = bf16lo(r.w); v[7] = bf16hi(r.w);
+  } else {
+    v[0] = __uint_as_float(r.x); v[1] = __uint_as_float(r.y);
+    v[2] = __uint_as_float(r.z); v[3] = __uint_as_float(r.w);
+  }
+}
+
+// VEC = channels per 16-byte vector (8 bf16 / 4 fp32); CH = vectors per lane;
+// U = voxel groups in flight per warp.
+template <typename T, int VEC, int CH, int U>
 __global__ void __launch_bounds__(kNormThreads) norm_silu_kernel(const T* __restrict__ x, T* y,
                                                                  const float* __restrict__ gamma,
                                                                  const float* __restrict__ beta,
                                                                  long nvox, int C, int L,
                                                                  float eps) {
+  extern __shared__ float sgb[];  // gamma [C], beta [C]
+  for (int i = threadIdx.x; i < C; i += blockDim.x) {
+    sgb[i] = gamma[i];
+    sgb[C + i] = beta[i];
+  }
+  __syncthreads();
   const int lane = threadIdx.x & 31;
-  const int sub = lane % L;                    // lane inside its voxel group
-  const int groups_per_warp = 32 / L;
-  const int nvec = C / VEC;                    // vectors per voxel
+  const int sub = lane % L;
+  const int gpw = 32 / L;                      // voxel groups per warp
+  const int nvec = C / VEC;
   const long warp_global = (static_cast<long>(blockIdx.x) * kNormThreads + threadIdx.x) >> 5;
   const long nwarps = (static_cast<long>(gridDim.x) * kNormThreads) >> 5;
   const float rootC = sqrtf(static_cast<float>(C));
+  const long step = nwarps * gpw;
 
-  float g[CH][VEC], b[CH][VEC];
-#pragma unroll
-  for (int k = 0; k < CH; ++k) {
-    const int vi = sub + k * L;
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      const int c = vi * VEC + e;
-      g[k][e] = (vi < nvec) ? gamma[c] : 0.0f;
-      b[k][e] = (vi < nvec) ? beta[c] : 0.0f;
-    }
-  }
-
-  // The loop bound is uniform across the warp (shuffles below need all lanes).
-  const long step = nwarps * groups_per_warp;
-  for (long wbase = warp_global * groups_per_warp; wbase < nvox; wbase += step * UNROLL) {
+  // The loop bound is uniform across the warp (the shuffles need all lanes).
+  for (long wbase = warp_global * gpw; wbase < nvox; wbase += step * U) {
     const long base = wbase + lane / L;
-    float v[UNROLL][CH][VEC];
-    float ss[UNROLL];
+    uint4 raw[U][CH];
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
+    for (int u = 0; u < U; ++u) {
       const long vox = base + u * step;
-      ss[u] = 0.0f;
 #pragma unroll
       for (int k = 0; k < CH; ++k) {
         const int vi = sub + k * L;
-        if (vox < nvox && vi < nvec) {
-          const uint4 raw = __ldg(reinterpret_cast<const uint4*>(x + vox * C) + vi);
-          if constexpr (VEC == 8) {
-            v[u][k][0] = bf16lo(raw.x); v[u][k][1] = bf16hi(raw.x);
-            v[u][k][2] = bf16lo(raw.y); v[u][k][3] = bf16hi(raw.y);
-            v[u][k][4] = bf16lo(raw.z); v[u][k][5] = bf16hi(raw.z);
-            v[u][k][6] = bf16lo(raw.w); v[u][k][7] = bf16hi(raw.w);
-          } else {
-            v[u][k][0] = __uint_as_float(raw.x); v[u][k][1] = __uint_as_float(raw.y);
-            v[u][k][2] = __uint_as_float(raw.z); v[u][k][3] = __uint_as_float(raw.w);
-          }
-        } else {
+        raw[u][k] = (vox < nvox && vi < nvec)
+                        ? __ldcs(reinterpret_cast<const uint4*>(x + vox * C) + vi)
+                        : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    float ss[U];
 #pragma unroll
-          for (int e = 0; e < VEC; ++e) v[u][k][e] = 0.0f;
-        }
+    for (int u = 0; u < U; ++u) {
+      ss[u] = 0.0f;
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) ss[u] = fmaf(v[u][k][e], v[u][k][e], ss[u]);
+      for (int k = 0; k < CH; ++k) {
+        float v[VEC];
+        unpack<VEC>(raw[u][k], v);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) ss[u] = fmaf(v[e], v[e], ss[u]);
       }
     }
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
+    for (int u = 0; u < U; ++u)
       for (int off = L >> 1; off > 0; off >>= 1) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], off);
-    }
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
+    for (int u = 0; u < U; ++u) {
       const long vox = base + u * step;
-      if (vox >= nvox) continue;
       const float r = rootC / fmaxf(sqrtf(ss[u]), eps);
 #pragma unroll
       for (int k = 0; k < CH; ++k) {
         const int vi = sub + k * L;
-        if (vi >= nvec) continue;
-        float o[VEC];
+        if (vox >= nvox || vi >= nvec) continue;
+        float v[VEC], o[VEC];
+        unpack<VEC>(raw[u][k], v);
+        const float* g = sgb + vi * VEC;
+        const float* b = sgb + C + vi * VEC;
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
-          const float s = v[u][k][e] * r * g[k][e] + b[k][e];
+          const float s = v[e] * r * g[e] + b[e];
           o[e] = (VEC == 8) ? silu_fast(s) : silu_exact(s);
         }
         uint4 w;
@@ -118,6 +122,24 @@ __global__ void __launch_bounds__(kNormThreads) norm_silu_kernel(const T* __rest
   }
 }
 
+template <typename T, int VEC, int CH, int U>
+cudaError_t launch_one(const T* x, T* y, const float* gamma, const float* beta, long nvox, int C,
+                       int L, float eps, int num_sms, cudaStream_t stream) {
+  auto kern = norm_silu_kernel<T, VEC, CH, U>;
+  const size_t smem = 2 * static_cast<size_t>(C) * sizeof(float);
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kNormThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  const long groups_per_block = (kNormThreads / 32) * (32 / L);
+  long blocks = (nvox + groups_per_block * U - 1) / (groups_per_block * U);
+  const long cap = static_cast<long>(num_sms) * per_sm;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  kern<<<static_cast<int>(blocks), kNormThreads, smem, stream>>>(x, y, gamma, beta, nvox, C, L, eps);
+  return cudaGetLastError();
+}
+
 template <typename T, int VEC>
 cudaError_t launch_impl(const T* x, T* y, const float* gamma, const float* beta, long nvox, int C,
                         float eps, int num_sms, cudaStream_t stream) {
@@ -125,24 +147,12 @@ cudaError_t launch_impl(const T* x, T* y, const float* gamma, const float* beta,
   int L = 1;
   while (L < nvec && L < 32) L <<= 1;
   const int ch = (nvec + L - 1) / L;
-  const long groups = nvox;
-  const long warps_needed = (groups * L + 31) / 32;
-  long blocks = (warps_needed + (kNormThreads / 32) - 1) / (kNormThreads / 32);
-  const long max_blocks = static_cast<long>(num_sms) * (2048 / kNormThreads);
-  if (blocks > max_blocks) blocks = max_blocks;
-  if (blocks < 1) blocks = 1;
-  const int grid = static_cast<int>(blocks);
-  if (ch == 1)
-    norm_silu_kernel<T, VEC, 1, 2><<<grid, kNormThreads, 0, stream>>>(x, y, gamma, beta, nvox, C, L, eps);
-  else if (ch == 2)
-    norm_silu_kernel<T, VEC, 2, 2><<<grid, kNormThreads, 0, stream>>>(x, y, gamma, beta, nvox, C, L, eps);
-  else if (ch <= 4)
-    norm_silu_kernel<T, VEC, 4, 1><<<grid, kNormThreads, 0, stream>>>(x, y, gamma, beta, nvox, C, L, eps);
-  else if (ch <= 8)
-    norm_silu_kernel<T, VEC, 8, 1><<<grid, kNormThreads, 0, stream>>>(x, y, gamma, beta, nvox, C, L, eps);
-  else
-    return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  // U * CH = 8 vectors (128 bytes) in flight per lane
+  if (ch == 1) return launch_one<T, VEC, 1, 8>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
+  if (ch == 2) return launch_one<T, VEC, 2, 4>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
+  if (ch <= 4) return launch_one<T, VEC, 4, 2>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
+  if (ch <= 8) return launch_one<T, VEC, 8, 1>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
