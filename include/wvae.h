@@ -207,6 +207,34 @@ WVAE_API wvae_status wvae_decode_trunk_timed(const void* const* packed, const fl
                                     size_t ws_bytes, void* const* events, int n_events,
                                     wvae_stream_t stream);
 
+/* ------------------------------------------------- res block, no allocation
+ * (No counterpart on the pages: this is a convenience of this library.)
+ *
+ * wvae_resblock for callers that cannot allocate device memory when they call
+ * it and have no workspace to pass in - for example a plugin run by a host
+ * engine that owns all device memory and hands its plugins none, or an
+ * application that forbids allocation after start-up so that its memory use
+ * is fixed and cannot fail mid-run.  Same arguments and result as
+ * wvae_resblock with dtype WVAE_BF16, but its scratch (the two activation
+ * tensors A1 and A2) lives in a static device array of 64 MiB inside this
+ * library, which every GPU that loads the library holds until the process
+ * exits.  It calls no allocator.
+ *   Size limit: round_up(T*H*W*cin*2, 256) + round_up(T*H*W*cout*2, 256)
+ *   <= 64 MiB (the value of wvae_resblock_workspace_bytes for bf16); larger
+ *   shapes return WVAE_ERR_WORKSPACE and enqueue nothing.
+ *   The first call on each device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   Every call on a device shares the one array, which keeps whatever the
+ *   last call left in it (nothing is read before it is written, so nothing
+ *   needs clearing).  Calls whose GPU work overlaps - two streams, two host
+ *   threads - race on it: serialise them.
+ */
+WVAE_API wvae_status wvae_resblock_noalloc(const void* x, void* y, int T, int H, int W, int cin,
+                                           int cout, const float* gamma1, const float* beta1,
+                                           const void* w1_packed, const float* gamma2,
+                                           const float* beta2, const void* w2_packed,
+                                           const void* wsc_packed, wvae_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -66,6 +66,7 @@ def load(path: str | None = None):
             "wvae_decode_trunk": (I, [ctypes.POINTER(V), ctypes.POINTER(V), V, V, I, I, I,
                                       ctypes.POINTER(I), I, V, S, V]),
             "wvae_decode_trunk_launches": (I, []),
+            "wvae_resblock_noalloc": (I, [V, V, I, I, I, I, I, V, V, V, V, V, V, V, V]),
             "wvae_decode_trunk_timed": (I, [ctypes.POINTER(V), ctypes.POINTER(V), V, V, I, I, I,
                                             ctypes.POINTER(I), I, V, S, ctypes.POINTER(V), I, V]),
         }

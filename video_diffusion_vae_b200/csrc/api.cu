@@ -714,4 +714,60 @@ wvae_status wvae_decode_trunk_timed(const void* const* packed, const float* cons
                            events, n_events, stream);
 }
 
+// ------------------------------------------------- res block, no allocation
+// Scratch for wvae_resblock_noalloc: its A1 and A2 activations.  A file-scope
+// device array, so callers that cannot allocate need not; it exists on every
+// GPU that loads this library until the process exits.  In host code the
+// array's name is not a device address: the address is looked up once per
+// device with cudaGetSymbolAddress and passed to the kernels.
+}  // extern "C"
+
+namespace wvae {
+namespace {
+constexpr size_t kNoAllocScratchBytes = 64ull << 20;
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device (set-up on the
+// first call per device, with that device current).
+wvae_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return WVAE_ERR_NO_DEVICE;
+  }
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return WVAE_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return WVAE_OK;
+}
+}  // namespace
+}  // namespace wvae
+
+extern "C" {
+
+wvae_status wvae_resblock_noalloc(const void* x, void* y, int T, int H, int W, int cin, int cout,
+                                  const float* gamma1, const float* beta1, const void* w1_packed,
+                                  const float* gamma2, const float* beta2, const void* w2_packed,
+                                  const void* wsc_packed, wvae_stream_t stream) {
+  if (T < 1 || H < 1 || W < 1 || cin < 1 || cout < 1) return WVAE_ERR_INVALID_ARG;
+  const size_t need = wvae_resblock_workspace_bytes(T, H, W, cin, cout, WVAE_BF16);
+  if (need > kNoAllocScratchBytes) return WVAE_ERR_WORKSPACE;
+  if (!x || !y || !gamma1 || !beta1 || !w1_packed || !gamma2 || !beta2 || !w2_packed)
+    return WVAE_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  wvae_status st = noalloc_scratch(&scratch);
+  if (st != WVAE_OK) return st;
+  return wvae_resblock(x, y, T, H, W, cin, cout, gamma1, beta1, w1_packed, gamma2, beta2,
+                       w2_packed, wsc_packed, WVAE_BF16, scratch, kNoAllocScratchBytes, stream);
+}
+
 }  // extern "C"
