@@ -108,13 +108,13 @@ PackedLayout packed_layout(int cout, int cin, int kt, int kh, int kw, wvae_dtype
 }
 
 // ------------------------------------------------------------ TMA descriptors
-bool encode_act(CUtensorMap* m, const void* base, int C, int W, int H, int T) {
+bool encode_act(CUtensorMap* m, const void* base, int C, int W, int H, int T, int box_h) {
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(W),
                         static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(C) * 2, static_cast<cuuint64_t>(C) * 2 * W,
                            static_cast<cuuint64_t>(C) * 2 * W * H};
   cuuint32_t box[4] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(kTileW),
-                       static_cast<cuuint32_t>(kTileH), 1};
+                       static_cast<cuuint32_t>(box_h), 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -173,10 +173,12 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
     p.BN = (L.cout_pad % 256 == 0) ? 256 : (L.cout_pad % 128 == 0 ? 128 : 16);
   }
   p.n_tiles = L.cout_pad / p.BN;
-  p.num_acc = p.BN <= 256 ? 2 : 1;
-  p.stages = conv_tc_stages_for(p.BN);
+  // Sub-tiles per CTA tile: S M=128 MMAs share each weight tile (see conv_tc.cu).
+  p.S = p.BN >= 256 ? 1 : (p.BN >= 128 ? 2 : 4);
+  p.num_acc = 2 * p.S * p.BN <= 512 ? 2 : 1;
+  p.stages = conv_tc_stages_for(p.BN, p.S);
   p.tiles_w = (a.W + kTileW - 1) / kTileW;
-  p.tiles_h = (a.H + kTileH - 1) / kTileH;
+  p.tiles_h = (a.H + kTileH * p.S - 1) / (kTileH * p.S);
   p.m_tiles = a.T * p.tiles_h * p.tiles_w;
   p.num_tiles = p.m_tiles * p.n_tiles;
   p.kblocks_main = L.taps * (a.cin_pad / kBK);
@@ -189,13 +191,14 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   p.ep = a.ep;
   p.err = d.err;
   const int box_rows = p.BN > 256 ? 256 : p.BN;
-  if (!encode_act(&p.tmA, a.x, a.cin_pad, a.W, a.H, a.T)) return WVAE_ERR_CUDA;
+  const int box_h = kTileH * p.S;
+  if (!encode_act(&p.tmA, a.x, a.cin_pad, a.W, a.H, a.T, box_h)) return WVAE_ERR_CUDA;
   if (!encode_weights(&p.tmB, a.packed, L.taps * a.cin_pad, L.cout_pad, box_rows))
     return WVAE_ERR_CUDA;
-  if (a.cache != nullptr && !encode_act(&p.tmC, a.cache, a.cin_pad, a.W, a.H, a.KT - 1))
+  if (a.cache != nullptr && !encode_act(&p.tmC, a.cache, a.cin_pad, a.W, a.H, a.KT - 1, box_h))
     return WVAE_ERR_CUDA;
   if (a.cin2_pad > 0) {
-    if (!encode_act(&p.tmA2, a.x2, a.cin2_pad, a.W, a.H, a.T)) return WVAE_ERR_CUDA;
+    if (!encode_act(&p.tmA2, a.x2, a.cin2_pad, a.W, a.H, a.T, box_h)) return WVAE_ERR_CUDA;
     if (!encode_weights(&p.tmB2, a.packed2, a.cin2_pad, L.cout_pad, box_rows)) return WVAE_ERR_CUDA;
   }
   const int grid = p.num_tiles < d.num_sms ? p.num_tiles : d.num_sms;

@@ -13,14 +13,19 @@
 // operands, fp32 accumulation; temporal caching: TensorRT-LLM issue #19309,
 // "Feature, motivation and proposed scope".)
 //
-// One CTA per SM, persistent over output tiles of 128 voxels (8 rows x 16
-// columns of one frame) x BN output channels.  Warp roles:
-//   warp 0      TMA producer: A box {64 ch, 16 w, 8 h, 1 t} + B box {64, BN}
+// One CTA per SM, persistent over output tiles of 8S rows x 16 columns of one
+// frame (S MMA sub-tiles of 128 voxels) x BN output channels.  Warp roles:
+//   warp 0      TMA producer: A box {64 ch, 16 w, 8S h, 1 t} + B box {64, BN}
 //               per K block into a ring of `stages` shared-memory stages;
-//   warp 1      MMA issuer: 4 x tcgen05.mma (M=128, N=BN<=256, K=16) per K
-//               block into a TMEM accumulator (two accumulators when BN <= 256,
-//               so the epilogue of tile i overlaps the main loop of tile i+1);
-//   warps 2..5  epilogue: one TMEM lane (= one output voxel) per thread.
+//   warp 1      MMA issuer: per K block, 4 K steps x S sub-tiles of
+//               tcgen05.mma (M=128, N=BN<=256, K=16) sharing the weight tile,
+//               into TMEM (two accumulators when 2 S BN <= 512, so the
+//               epilogue of tile i overlaps the main loop of tile i+1);
+//   warps 2..5  epilogue: one TMEM lane (= one output voxel per sub-tile) per
+//               thread.
+// tcgen05.mma issue runs nearly in step with execution, so every cycle the
+// issuing thread spends waiting on a barrier is a tensor-pipe bubble: S
+// sub-tiles per weight tile put S times more MMA work behind each wait.
 // The epilogue adds bias (and residual), and may emit the raw result (fp32 or
 // bf16, optionally 2x-upsampled), the next layer's SiLU(norm(.)) activation
 // (the whole channel vector of the voxel is in the thread's TMEM lane, so the
@@ -57,7 +62,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw, const ConvParams& p) {
   uint32_t base = smem_u32(raw);
   uint32_t pad = (1024u - (base & 1023u)) & 1023u;
   uint8_t* al = raw + pad;
-  s.a_bytes = kBM * kBK * 2;
+  s.a_bytes = static_cast<uint32_t>(kBM) * p.S * kBK * 2;
   s.stage_bytes = s.a_bytes + static_cast<uint32_t>(p.BN) * kBK * 2;
   s.stages = al;
   uint8_t* ctrl = al + p.stages * s.stage_bytes;
@@ -100,7 +105,7 @@ __device__ void producer(const ConvParams& p, const Smem& s) {
   bool aborted = false;
   for (int tile = blockIdx.x; tile < p.num_tiles && !aborted; tile += gridDim.x) {
     const TileCoord tc = decode_tile(p, tile);
-    const int h0 = tc.th * kTileH, w0 = tc.tw * kTileW;
+    const int h0 = tc.th * kTileH * p.S, w0 = tc.tw * kTileW;
     for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
       const uint32_t st = it % p.stages;
       const uint32_t ph = (it / p.stages) & 1u;
@@ -147,12 +152,29 @@ __device__ void producer(const ConvParams& p, const Smem& s) {
 }
 
 // ----------------------------------------------------------------------- MMA
+__device__ __noinline__ bool mma_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                           unsigned* err) {
+  return mbar_wait_bounded(bar, parity, abort_flag, err, DEVERR_TIMEOUT_MMA);
+}
+
+// S sub-tiles and HALVES weight halves are compile-time so the issue loop is
+// fully unrolled: the thread must hand the next MMA to the tensor core as soon
+// as it can take it.
+template <int S, int HALVES>
 __device__ void mma_issuer(const ConvParams& p, const Smem& s, uint32_t tmem_base) {
   const int n_inst = p.BN > 256 ? 256 : p.BN;
-  const int halves = p.BN > 256 ? 2 : 1;
   const uint32_t idesc = umma_idesc_bf16(kBM, n_inst);
-  const uint32_t b_half_bytes = 256u * kBK * 2;
-  uint32_t it = 0, ai = 0;
+  // Descriptors of stage 0; the start field counts 16-byte units: stage st
+  // adds stage_bytes / 16, sub-tile s adds 16 KB / 16, K step k adds 32 B / 16
+  // and the second weight half 32 KB / 16.
+  const uint64_t adesc0 = umma_desc_sw128(smem_u32(s.stages));
+  const uint64_t bdesc0 = umma_desc_sw128(smem_u32(s.stages) + s.a_bytes);
+  const uint32_t stage_step = s.stage_bytes >> 4;
+  const uint32_t sub_step = (static_cast<uint32_t>(kBM) * 128u) >> 4;
+  const uint32_t full0 = smem_u32(&s.full[0]), empty0 = smem_u32(&s.empty[0]);
+  const uint32_t bn = static_cast<uint32_t>(p.BN);
+  const uint32_t acc_cols = static_cast<uint32_t>(S) * bn;
+  uint32_t st = 0, ph = 0, ai = 0;
   bool aborted = false;
   for (int tile = blockIdx.x; tile < p.num_tiles && !aborted; tile += gridDim.x, ++ai) {
     const uint32_t acc = ai % p.num_acc;
@@ -163,27 +185,32 @@ __device__ void mma_issuer(const ConvParams& p, const Smem& s, uint32_t tmem_bas
       break;
     }
     tc_fence_after();
-    const uint32_t d_tmem = tmem_base + acc * 256u;
-    for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
-      const uint32_t st = it % p.stages;
-      const uint32_t ph = (it / p.stages) & 1u;
-      if (!mbar_wait_bounded(smem_u32(&s.full[st]), ph, s.abort_flag, p.err,
-                             DEVERR_TIMEOUT_MMA)) {
+    const uint32_t d_tmem = tmem_base + acc * acc_cols;
+    for (int kb = 0; kb < p.kblocks; ++kb) {
+      const uint32_t bar = full0 + st * 8u;
+      if (!mbar_try_wait(bar, ph) && !mma_wait_slow(bar, ph, s.abort_flag, p.err)) {
         aborted = true;
         break;
       }
       tc_fence_after();
-      const uint32_t a_addr = smem_u32(s.stages + st * s.stage_bytes);
-      const uint32_t b_addr = a_addr + s.a_bytes;
+      const uint64_t a_st = adesc0 + st * stage_step;
+      const uint64_t b_st = bdesc0 + st * stage_step;
 #pragma unroll
       for (int k = 0; k < kBK / 16; ++k) {
-        const uint64_t adesc = umma_desc_sw128(a_addr + k * 32);
-        for (int hf = 0; hf < halves; ++hf) {
-          const uint64_t bdesc = umma_desc_sw128(b_addr + hf * b_half_bytes + k * 32);
-          umma_bf16(d_tmem + hf * 256u, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+        const uint32_t accumulate = (kb | k) != 0 ? 1u : 0u;
+#pragma unroll
+        for (int sub = 0; sub < S; ++sub) {
+          const uint64_t a_k = a_st + sub * sub_step + 2u * k;
+          const uint32_t d_sub = d_tmem + static_cast<uint32_t>(sub) * bn;
+          umma_bf16(d_sub, a_k, b_st + 2u * k, idesc, accumulate);
+          if (HALVES == 2) umma_bf16(d_sub + 256u, a_k, b_st + 2048u + 2u * k, idesc, accumulate);
         }
       }
-      umma_commit(smem_u32(&s.empty[st]));
+      umma_commit(empty0 + st * 8u);
+      if (++st == static_cast<uint32_t>(p.stages)) {
+        st = 0;
+        ph ^= 1u;
+      }
     }
     if (aborted) break;
     umma_commit(smem_u32(&s.tfull[acc]));
@@ -310,7 +337,7 @@ __device__ __forceinline__ void emit_chunk(const ConvParams& p, const Smem& s, i
 #pragma unroll
     for (int j = 0; j < NC; ++j) {
       const float sv = v[j] * rs * s.gamma[n0 + c0 + j] + s.beta[n0 + c0 + j];
-      a[j] = sv * __frcp_rn(1.0f + __expf(-sv));
+      a[j] = silu_fast(sv);
     }
     store_bf16<NC>(ep.act + vox * p.cout + n0 + c0, a);
   }
@@ -349,40 +376,43 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
     if (!ok) break;
     tc_fence_after();
     const TileCoord tc = decode_tile(p, tile);
-    const int h = tc.th * kTileH + hl, w = tc.tw * kTileW + wl;
-    const bool valid = h < p.H && w < p.W;
-    const size_t vox = (static_cast<size_t>(tc.t) * p.H + h) * p.W + w;
     const int n0 = tc.n_tile * p.BN;
-    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * 256u;
-
-    float rs = 1.0f;
-    if (p.ep.act != nullptr) {
-      float ss = 0.0f;
+    for (int sub = 0; sub < p.S; ++sub) {
+      const int h = (tc.th * p.S + sub) * kTileH + hl, w = tc.tw * kTileW + wl;
+      const bool valid = h < p.H && w < p.W;
+      const size_t vox = (static_cast<size_t>(tc.t) * p.H + h) * p.W + w;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             acc * static_cast<uint32_t>(p.S * p.BN) +
+                             static_cast<uint32_t>(sub * p.BN);
+      float rs = 1.0f;
+      if (p.ep.act != nullptr) {
+        float ss = 0.0f;
+        int c0 = 0;
+        for (; c0 + 32 <= p.BN; c0 += 32) {
+          float v[32];
+          result_chunk<32>(p, s, taddr, c0, n0, valid, vox, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
+        }
+        if (c0 < p.BN) {
+          float v[16];
+          result_chunk<16>(p, s, taddr, c0, n0, valid, vox, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) ss = fmaf(v[j], v[j], ss);
+        }
+        rs = rootC / fmaxf(sqrtf(ss), p.ep.eps);
+      }
       int c0 = 0;
       for (; c0 + 32 <= p.BN; c0 += 32) {
         float v[32];
         result_chunk<32>(p, s, taddr, c0, n0, valid, vox, v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
+        if (valid) emit_chunk<32>(p, s, c0, n0, tc, h, w, vox, rs, v);
       }
       if (c0 < p.BN) {
         float v[16];
         result_chunk<16>(p, s, taddr, c0, n0, valid, vox, v);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) ss = fmaf(v[j], v[j], ss);
+        if (valid) emit_chunk<16>(p, s, c0, n0, tc, h, w, vox, rs, v);
       }
-      rs = rootC / fmaxf(sqrtf(ss), p.ep.eps);
-    }
-    int c0 = 0;
-    for (; c0 + 32 <= p.BN; c0 += 32) {
-      float v[32];
-      result_chunk<32>(p, s, taddr, c0, n0, valid, vox, v);
-      if (valid) emit_chunk<32>(p, s, c0, n0, tc, h, w, vox, rs, v);
-    }
-    if (c0 < p.BN) {
-      float v[16];
-      result_chunk<16>(p, s, taddr, c0, n0, valid, vox, v);
-      if (valid) emit_chunk<16>(p, s, c0, n0, tc, h, w, vox, rs, v);
     }
     tc_fence_before();
     mbar_arrive(smem_u32(&s.tempty[acc]));
@@ -432,7 +462,16 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
   if (warp == 0) {
     if (lane == 0) producer(p, s);
   } else if (warp == 1) {
-    if (lane == 0) mma_issuer(p, s, tmem_base);
+    if (lane == 0) {
+      if (p.BN > 256)
+        mma_issuer<1, 2>(p, s, tmem_base);
+      else if (p.S == 1)
+        mma_issuer<1, 1>(p, s, tmem_base);
+      else if (p.S == 2)
+        mma_issuer<2, 1>(p, s, tmem_base);
+      else
+        mma_issuer<4, 1>(p, s, tmem_base);
+    }
   } else {
     epilogue(p, s, tmem_base, warp, lane);
   }
@@ -448,20 +487,23 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
 
 }  // namespace
 
-size_t conv_tc_smem_bytes(int BN, int stages) {
-  const size_t stage = static_cast<size_t>(kBM) * kBK * 2 + static_cast<size_t>(BN) * kBK * 2;
+size_t conv_tc_smem_bytes(int BN, int S, int stages) {
+  const size_t stage = static_cast<size_t>(kBM) * S * kBK * 2 + static_cast<size_t>(BN) * kBK * 2;
   return 1024 + stages * stage + kCtrlBytes;
 }
 
-int conv_tc_stages_for(int BN) {
+int conv_tc_stages_for(int BN, int S) {
   const size_t limit = 232448;  // 227 KB opt-in dynamic shared memory per block
   int st = kMaxStages;
-  while (st > 2 && conv_tc_smem_bytes(BN, st) > limit) --st;
+  while (st > 2 && conv_tc_smem_bytes(BN, S, st) > limit) --st;
   return st;
 }
 
 cudaError_t launch_conv_tc(const ConvParams& p, int grid, cudaStream_t stream) {
-  const size_t smem = conv_tc_smem_bytes(p.BN, p.stages);
+  // Every CTA allocates all 512 TMEM columns, so exactly one may live on an SM:
+  // ask for more than half of the SM's shared memory even when the ring is small.
+  size_t smem = conv_tc_smem_bytes(p.BN, p.S, p.stages);
+  if (smem < 120 * 1024) smem = 120 * 1024;
   cudaError_t e = cudaFuncSetAttribute(conv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;

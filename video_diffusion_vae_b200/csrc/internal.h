@@ -10,8 +10,10 @@
 namespace wvae {
 
 // ----------------------------------------------------------- conv (tcgen05)
-// Output tile: 128 voxels of one frame, 8 rows x 16 columns; K block: 64
-// input channels of one tap.
+// MMA sub-tile: 128 voxels of one frame, 8 rows x 16 columns (MMA row m =
+// 16 * row + column).  A CTA tile stacks S sub-tiles (8S rows x 16 columns),
+// whose S M=128 MMAs share each weight tile.  K block: 64 input channels of
+// one tap.
 constexpr int kTileH = 8;
 constexpr int kTileW = 16;
 constexpr int kBM = kTileH * kTileW;  // 128
@@ -36,10 +38,10 @@ struct ConvEpilogue {
 };
 
 struct ConvParams {
-  CUtensorMap tmA;   // main input, bf16 [T][H][W][cin_pad], box {64, 16, 8, 1}
+  CUtensorMap tmA;   // main input, bf16 [T][H][W][cin_pad], box {64, 16, 8S, 1}
   CUtensorMap tmB;   // main weights, bf16 [cout_pad][taps * cin_pad], box {64, <=256}
-  CUtensorMap tmC;   // cached frames, bf16 [KT-1][H][W][cin_pad] (has_cache)
-  CUtensorMap tmA2;  // shortcut input, bf16 [T][H][W][cin2_pad] (cin2_pad > 0)
+  CUtensorMap tmC;   // cached frames, bf16 [KT-1][H][W][cin_pad], box as tmA (has_cache)
+  CUtensorMap tmA2;  // shortcut input, bf16 [T][H][W][cin2_pad], box as tmA (cin2_pad > 0)
   CUtensorMap tmB2;  // shortcut weights, bf16 [cout_pad][cin2_pad]
   int T, H, W;
   int cin_pad, cin2_pad;
@@ -47,15 +49,16 @@ struct ConvParams {
   int KT, KH, KW;
   int has_cache;
   int BN, n_tiles;
-  int tiles_w, tiles_h, m_tiles, num_tiles;
+  int S;             // MMA sub-tiles per CTA tile; S * BN <= 512 TMEM columns
+  int tiles_w, tiles_h, m_tiles, num_tiles;  // CTA tiles of 8S rows x 16 columns
   int stages, num_acc;
   int kblocks_main, kblocks;
   ConvEpilogue ep;
   unsigned* err;
 };
 
-size_t conv_tc_smem_bytes(int BN, int stages);
-int conv_tc_stages_for(int BN);
+size_t conv_tc_smem_bytes(int BN, int S, int stages);
+int conv_tc_stages_for(int BN, int S);
 cudaError_t launch_conv_tc(const ConvParams& p, int grid, cudaStream_t stream);
 
 // ------------------------------------------------------------ fp32 direct conv

@@ -13,8 +13,9 @@
 // channels), so a warp's accesses to a voxel are one contiguous, fully
 // coalesced run.  Each warp first issues the loads of U voxel groups (kept
 // packed in registers), then reduces the sums of squares with shuffles inside
-// each group and writes the results; gamma/beta sit in shared memory.  The grid
-// is persistent: exactly the blocks that fit on the GPU at once.
+// each group and writes the results.  A lane's channels never change, so its
+// gamma/beta live in registers for the whole kernel.  The grid is persistent:
+// exactly the blocks that fit on the GPU at once.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -24,7 +25,6 @@ namespace {
 
 constexpr int kNormThreads = 256;
 
-__device__ __forceinline__ float silu_fast(float s) { return s * __frcp_rn(1.0f + __expf(-s)); }
 __device__ __forceinline__ float silu_exact(float s) { return s / (1.0f + expf(-s)); }
 
 template <int VEC>
@@ -41,21 +41,25 @@ __device__ __forceinline__ void unpack(const uint4& r, float (&v)[VEC]) {
 // VEC = channels per 16-byte vector (8 bf16 / 4 fp32); CH = vectors per lane;
 // U = voxel groups in flight per warp.
 template <typename T, int VEC, int CH, int U>
-__global__ void __launch_bounds__(kNormThreads) norm_silu_kernel(const T* __restrict__ x, T* y,
+__global__ void __launch_bounds__(kNormThreads, (VEC == 8 && CH <= 4) ? 3 : 2) norm_silu_kernel(const T* __restrict__ x, T* y,
                                                                  const float* __restrict__ gamma,
                                                                  const float* __restrict__ beta,
                                                                  long nvox, int C, int L,
                                                                  float eps) {
-  extern __shared__ float sgb[];  // gamma [C], beta [C]
-  for (int i = threadIdx.x; i < C; i += blockDim.x) {
-    sgb[i] = gamma[i];
-    sgb[C + i] = beta[i];
-  }
-  __syncthreads();
   const int lane = threadIdx.x & 31;
   const int sub = lane % L;
   const int gpw = 32 / L;                      // voxel groups per warp
   const int nvec = C / VEC;
+  float g[CH][VEC], b[CH][VEC];
+#pragma unroll
+  for (int k = 0; k < CH; ++k) {
+    const int vi = sub + k * L;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      g[k][e] = vi < nvec ? __ldg(gamma + vi * VEC + e) : 0.0f;
+      b[k][e] = vi < nvec ? __ldg(beta + vi * VEC + e) : 0.0f;
+    }
+  }
   const long warp_global = (static_cast<long>(blockIdx.x) * kNormThreads + threadIdx.x) >> 5;
   const long nwarps = (static_cast<long>(gridDim.x) * kNormThreads) >> 5;
   const float rootC = sqrtf(static_cast<float>(C));
@@ -101,11 +105,9 @@ __global__ void __launch_bounds__(kNormThreads) norm_silu_kernel(const T* __rest
         if (vox >= nvox || vi >= nvec) continue;
         float v[VEC], o[VEC];
         unpack<VEC>(raw[u][k], v);
-        const float* g = sgb + vi * VEC;
-        const float* b = sgb + C + vi * VEC;
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
-          const float s = v[e] * r * g[e] + b[e];
+          const float s = v[e] * r * g[k][e] + b[k][e];
           o[e] = (VEC == 8) ? silu_fast(s) : silu_exact(s);
         }
         uint4 w;
@@ -126,7 +128,7 @@ template <typename T, int VEC, int CH, int U>
 cudaError_t launch_one(const T* x, T* y, const float* gamma, const float* beta, long nvox, int C,
                        int L, float eps, int num_sms, cudaStream_t stream) {
   auto kern = norm_silu_kernel<T, VEC, CH, U>;
-  const size_t smem = 2 * static_cast<size_t>(C) * sizeof(float);
+  const size_t smem = 0;
   int per_sm = 0;
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kNormThreads, smem);
   if (e != cudaSuccess) return e;
@@ -147,10 +149,10 @@ cudaError_t launch_impl(const T* x, T* y, const float* gamma, const float* beta,
   int L = 1;
   while (L < nvec && L < 32) L <<= 1;
   const int ch = (nvec + L - 1) / L;
-  // U * CH = 8 vectors (128 bytes) in flight per lane
-  if (ch == 1) return launch_one<T, VEC, 1, 8>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
-  if (ch == 2) return launch_one<T, VEC, 2, 4>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
-  if (ch <= 4) return launch_one<T, VEC, 4, 2>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
+  // U * CH <= 4 vectors (64 bytes) in flight per lane keeps 3 blocks of 256 per SM
+  if (ch == 1) return launch_one<T, VEC, 1, 4>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
+  if (ch == 2) return launch_one<T, VEC, 2, 2>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
+  if (ch <= 4) return launch_one<T, VEC, 4, 1>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
   if (ch <= 8) return launch_one<T, VEC, 8, 1>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
   return cudaErrorInvalidValue;
 }

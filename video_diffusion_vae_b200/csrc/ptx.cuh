@@ -189,6 +189,17 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
 }
 
 // ------------------------------------------------------------ numeric helpers
+// Single-instruction approximate reciprocal (rcp.approx.ftz): 1/inf -> 0.
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+// SiLU(s) = s * sigmoid(s) with the SFU exp and reciprocal (bf16 outputs);
+// s -> -inf gives -0, s -> +inf gives s.
+__device__ __forceinline__ float silu_fast(float s) {
+  return s * rcp_approx(1.0f + __expf(-s));
+}
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
