@@ -174,7 +174,7 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   }
   p.n_tiles = L.cout_pad / p.BN;
   // Sub-tiles per CTA tile: S M=128 MMAs share each weight tile (see conv_tc.cu).
-  p.S = p.BN >= 256 ? 1 : (p.BN >= 128 ? 2 : 4);
+  p.S = p.BN >= 512 ? 1 : (p.BN >= 128 ? 2 : 4);
   p.num_acc = 2 * p.S * p.BN <= 512 ? 2 : 1;
   p.stages = conv_tc_stages_for(p.BN, p.S);
   p.tiles_w = (a.W + kTileW - 1) / kTileW;
