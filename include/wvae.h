@@ -157,9 +157,21 @@ WVAE_API wvae_status wvae_resblock(const void* x, void* y, int T, int H, int W, 
 /* -------------------------------------------------- upsample + 3x3 conv
  * y[t] = conv3x3( nearest2x(x[t]) ) + bias, per frame, zero border of 1 at the
  * upsampled resolution; u[2h+i, 2w+j] = x[h, w].
+ * bf16: computed without materialising u, as four 2x2 "phase" convs on x
+ * (the FastVideo README's "phase" weight transform, section "Use"): output
+ * pixel (2h+p, 2w+q) reads x rows h+p-1, h+p and columns w+q-1, w+q with the
+ * 3x3 taps that land on them summed (in fp32, rounded once to bf16) by
+ * wvae_prepack_upsample_conv.  fp32: the reference path materialises u in the
+ * workspace and runs the fp32 (1,3,3) conv.
+ *   w: PyTorch [cout][cin][1][3][3] (device, fp32 or bf16); bias fp32 [cout] or NULL.
  *   x: [T][H][W][cin], y: [T][2H][2W][cout] in dtype.
- *   packed_w: (cout, cin, 1, 3, 3).   workspace: see the _bytes query.
+ *   packed_w: from wvae_prepack_upsample_conv for (cout, cin, dtype).
+ *   workspace: wvae_upsample_conv_workspace_bytes(...) bytes (0 for bf16).
  */
+WVAE_API size_t wvae_upsample_conv_packed_bytes(int cout, int cin, wvae_dtype dtype);
+WVAE_API wvae_status wvae_prepack_upsample_conv(const void* w, wvae_dtype w_dtype, const float* bias,
+                                       int cout, int cin, wvae_dtype dtype, void* packed,
+                                       size_t packed_bytes, wvae_stream_t stream);
 WVAE_API size_t wvae_upsample_conv_workspace_bytes(int T, int H, int W, int cin, wvae_dtype dtype);
 WVAE_API wvae_status wvae_upsample_conv(const void* x, void* y, int T, int H, int W, int cin, int cout,
                                const void* packed_w, wvae_dtype dtype, void* workspace,
@@ -176,8 +188,8 @@ WVAE_API wvae_status wvae_upsample_conv(const void* x, void* y, int T, int H, in
  *     64 and <= 256 or == 512.
  *   packed: host array of 21 device pointers, in forward order:
  *     [0] conv_in (C0, 48, 3,3,3); per stage s, per block b: conv1 (Cs, Cs, 3,3,3),
- *     conv2 (Cs, Cs, 3,3,3); then for s < 3 the upsample conv (C(s+1), Cs, 1,3,3);
- *     [20] head (12, C3, 3,3,3).
+ *     conv2 (Cs, Cs, 3,3,3) (wvae_prepack_conv); then for s < 3 the upsample conv
+ *     (C(s+1), Cs) from wvae_prepack_upsample_conv; [20] head (12, C3, 3,3,3).
  *   norms: host array of 34 device pointers (fp32), gamma then beta for each norm in
  *     forward order: per stage, per block: norm1, norm2; then norm_out.
  *   workspace: wvae_decode_trunk_workspace_bytes(T, H, W, widths) bytes.

@@ -20,7 +20,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     declared = B.header_symbols()
-    assert len(declared) == 17
+    assert len(declared) == 19
     out = subprocess.check_output(["nm", "-D", "--defined-only", B.LIB_PATH], text=True)
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
     missing = [s for s in declared if s not in exported]
@@ -56,7 +56,10 @@ def test_workspace_sizes(lib):
     assert lib.wvae_resblock_workspace_bytes(4, 176, 312, 256, 256, B.BF16) == 2 * nv * 256 * 2
     assert lib.wvae_causal_conv3d_workspace_bytes(4, 88, 156, 512, 0, B.BF16) == 0
     assert lib.wvae_causal_conv3d_workspace_bytes(4, 88, 156, 512, 1, B.BF16) == 4 * 88 * 156 * 512 * 2
-    assert lib.wvae_upsample_conv_workspace_bytes(4, 88, 156, 512, B.BF16) == 4 * 176 * 312 * 512 * 2
+    assert lib.wvae_upsample_conv_workspace_bytes(4, 88, 156, 512, B.BF16) == 0      # phase convs
+    assert lib.wvae_upsample_conv_workspace_bytes(4, 88, 156, 512, B.F32) == 4 * 176 * 312 * 512 * 4
+    # four 2x2 phase kernels: [cout_pad][16][cin_pad] bf16 + bias
+    assert lib.wvae_upsample_conv_packed_bytes(256, 512, B.BF16) == 256 * 16 * 512 * 2 + 256 * 4
     assert lib.wvae_decode_trunk_workspace_bytes(4, 44, 78, None) > 4 * 352 * 624 * 128 * 4
     assert lib.wvae_decode_trunk_workspace_bytes(0, 44, 78, None) == 0
 

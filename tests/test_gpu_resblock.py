@@ -55,14 +55,54 @@ def test_resblock_full_size_sampled(cout):
     assert B.device_error() == 0
 
 
-@pytest.mark.parametrize("cin,cout,H,W", [(128, 64, 6, 10), (64, 128, 5, 9), (512, 256, 4, 8)])
+@pytest.mark.parametrize("cin,cout,H,W", [(128, 64, 6, 10), (64, 128, 5, 9), (512, 256, 4, 8),
+                                          (256, 128, 9, 21)])
 def test_upsample_conv(cin, cout, H, W):
+    """Nearest 2x + 3x3 conv via the four phase kernels vs the oracle's dense definition."""
     g = torch.Generator().manual_seed(cin)
     x = synth.normal(g, (cin, 2, H, W))
     w, b = synth.conv_params(g, cout, cin, 1, 3, 3)
-    pk = B.prepack_conv(w.cuda().bfloat16(), b.cuda())
+    pk = B.prepack_upsample_conv(w.cuda().bfloat16(), b.cuda())
     y = B.upsample_conv(to_cl(x), pk)
+    assert y.shape == (2, 2 * H, 2 * W, cout)
     assert_close(from_cl(y), O.upsample_conv(x, w, b), torch.bfloat16, "upsample conv")
+
+
+def test_upsample_conv_f32():
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(64, 2, 5, 7, generator=g)
+    w = torch.randn(32, 64, 1, 3, 3, generator=g) / 24.0
+    b = 0.1 * torch.randn(32, generator=g)
+    pk = B.prepack_upsample_conv(w.cuda(), b.cuda(), torch.float32)
+    y = B.upsample_conv(to_cl(x, torch.float32), pk)
+    assert_close(from_cl(y), O.upsample_conv(x, w, b), torch.float32, "upsample conv fp32")
+
+
+def test_upsample_conv_full_size_sampled():
+    """The trunk's 512 -> 256 upsample conv at [512, 4, 88, 156] -> [256, 4, 176, 312], sampled."""
+    g = torch.Generator().manual_seed(21)
+    x = synth.normal(g, (512, 4, 88, 156))
+    w, b = synth.conv_params(g, 256, 512, 1, 3, 3)
+    pk = B.prepack_upsample_conv(w.cuda().bfloat16(), b.cuda())
+    y = B.upsample_conv(to_cl(x), pk)
+    torch.cuda.synchronize()
+    yc = y.float().cpu()
+    pts = sample_voxels(4, 176, 312, 24, seed=4)
+    got = np.stack([yc[t, h, ww].double().numpy() for (t, h, ww) in pts], 1)
+    ref = []
+    for (t, h, ww) in pts:
+        # the output pixel depends on a 2x2 low-res window: crop, upsample, conv, read the centre
+        h0, w0 = max(0, h // 2 - 1), max(0, ww // 2 - 1)
+        h1, w1 = min(88, h // 2 + 2), min(156, ww // 2 + 2)
+        crop = x[:, t:t + 1, h0:h1, w0:w1]
+        yy = O.upsample_conv(crop, w, b)
+        hb, wb = h - 2 * h0, ww - 2 * w0
+        edge_ok = (h0 == 0 or hb >= 1) and (h1 == 88 or hb <= 2 * (h1 - h0) - 2) and \
+                  (w0 == 0 or wb >= 1) and (w1 == 156 or wb <= 2 * (w1 - w0) - 2)
+        assert edge_ok
+        ref.append(yy[:, 0, hb, wb])
+    assert_close(got, np.stack(ref, 1), torch.bfloat16, "upsample conv full size")
+    assert B.device_error() == 0
 
 
 def _trunk_case(T, H, W, widths, zc=48, seed=0):

@@ -60,6 +60,8 @@ def load(path: str | None = None):
             "wvae_causal_conv3d": (I, [V, V, V, I, I, I, I, I, I, I, I, V, V, V, V, I, V, S, V]),
             "wvae_resblock_workspace_bytes": (S, [I, I, I, I, I, I]),
             "wvae_resblock": (I, [V, V, I, I, I, I, I, V, V, V, V, V, V, V, I, V, S, V]),
+            "wvae_upsample_conv_packed_bytes": (S, [I, I, I]),
+            "wvae_prepack_upsample_conv": (I, [V, I, V, I, I, I, V, S, V]),
             "wvae_upsample_conv_workspace_bytes": (S, [I, I, I, I, I]),
             "wvae_upsample_conv": (I, [V, V, I, I, I, I, I, V, I, V, S, V]),
             "wvae_decode_trunk_workspace_bytes": (S, [I, I, I, ctypes.POINTER(I)]),
@@ -180,6 +182,22 @@ def prepack_conv(w, bias=None, dtype=torch.bfloat16) -> PackedConv:
     return PackedConv(blob, cout, cin, (kt, kh, kw), dt)
 
 
+def prepack_upsample_conv(w, bias=None, dtype=torch.bfloat16) -> PackedConv:
+    """Upsample-conv weights [Cout, Cin, 1, 3, 3] -> the four 2x2 phase kernels (bf16)
+    or the plain fp32 packing (fp32 reference path)."""
+    _cuda(w, "w")
+    cout, cin, kt, kh, kw = w.shape
+    if (kt, kh, kw) != (1, 3, 3):
+        raise ValueError("upsample conv weights must be [Cout, Cin, 1, 3, 3]")
+    dt = BF16 if dtype == torch.bfloat16 else F32
+    n = load().wvae_upsample_conv_packed_bytes(cout, cin, dt)
+    blob = torch.empty(n, dtype=torch.uint8, device=w.device)
+    b = None if bias is None else _f32vec(bias, cout, "bias")
+    _check("wvae_prepack_upsample_conv", load().wvae_prepack_upsample_conv(
+        _ptr(w), _dt(w), _ptr(b), cout, cin, dt, _ptr(blob), n, _stream()))
+    return PackedConv(blob, cout, cin, (1, 3, 3), dt)
+
+
 # ---------------------------------------------------------------- causal conv
 def causal_conv3d(x, packed: PackedConv, cache=None, norm=None, residual=None, out=None):
     """Causal conv of x [T, H, W, Cin]; norm = (gamma, beta) applies SiLU(norm(x)) first."""
@@ -250,7 +268,7 @@ def upsample_conv(x, packed: PackedConv, out=None):
         _cuda(out, "out", x.dtype, (T, 2 * H, 2 * W, cout))
     lib = load()
     nws = lib.wvae_upsample_conv_workspace_bytes(T, H, W, cin, dt)
-    ws = _workspace(nws, x.device)
+    ws = _workspace(nws, x.device) if nws else None
     _check("wvae_upsample_conv", lib.wvae_upsample_conv(
         _ptr(x), _ptr(y), T, H, W, cin, cout, packed.ptr(), dt, _ptr(ws), nws, _stream()))
     return y
@@ -272,7 +290,8 @@ class PackedTrunk:
                 self.norms += [f(bp["gamma1"]), f(bp["beta1"]), f(bp["gamma2"]), f(bp["beta2"])]
                 self.convs += [pk(bp["w1"], bp["b1"]), pk(bp["w2"], bp["b2"])]
             if st["up"] is not None:
-                self.convs.append(pk(*st["up"]))
+                wu, bu = st["up"]
+                self.convs.append(prepack_upsample_conv(wu.to(dev, torch.bfloat16).contiguous(), f(bu)))
         hp = params["head"]
         self.norms += [f(hp["gamma"]), f(hp["beta"])]
         self.convs.append(pk(hp["w"], hp["b"]))

@@ -144,12 +144,20 @@ struct TcConv {
   int cin2_pad = 0;
   const void* packed2 = nullptr;
   int T = 0, H = 0, W = 0;
+  int phases = 1;            // 4: upsample-conv phase mode (packed by prepack_upsample)
   ConvEpilogue ep{};
 };
 
 wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   static_assert(sizeof(ConvParams) < 4000, "kernel parameter space");
-  const PackedLayout L = packed_layout(a.cout, a.cin_pad, a.KT, a.KH, a.KW, WVAE_BF16);
+  if (a.phases == 4) {
+    a.KT = 1;
+    a.KH = 2;
+    a.KW = 2;
+  }
+  // phase mode packs 4 phases x 4 taps along K
+  const PackedLayout L = a.phases == 4 ? packed_layout(a.cout, a.cin_pad, 1, 4, 4, WVAE_BF16)
+                                       : packed_layout(a.cout, a.cin_pad, a.KT, a.KH, a.KW, WVAE_BF16);
   ConvParams p;
   std::memset(&p, 0, sizeof(p));
   p.T = a.T;
@@ -162,6 +170,7 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   p.KT = a.KT;
   p.KH = a.KH;
   p.KW = a.KW;
+  p.phases = a.phases;
   p.has_cache = a.cache != nullptr;
   const bool need_all_channels = a.ep.act != nullptr;
   if (L.cout_pad <= 256) {
@@ -180,8 +189,8 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   p.tiles_w = (a.W + kTileW - 1) / kTileW;
   p.tiles_h = (a.H + kTileH * p.S - 1) / (kTileH * p.S);
   p.m_tiles = a.T * p.tiles_h * p.tiles_w;
-  p.num_tiles = p.m_tiles * p.n_tiles;
-  p.kblocks_main = L.taps * (a.cin_pad / kBK);
+  p.num_tiles = p.m_tiles * p.phases * p.n_tiles;
+  p.kblocks_main = a.KT * a.KH * a.KW * (a.cin_pad / kBK);
   p.kblocks = p.kblocks_main + a.cin2_pad / kBK;
   a.ep.bias = reinterpret_cast<const float*>(static_cast<const char*>(a.packed) + L.bias_off);
   if (a.packed2 != nullptr) {
@@ -468,8 +477,37 @@ wvae_status wvae_resblock(const void* x, void* y, int T, int H, int W, int cin, 
 }
 
 // ------------------------------------------------------ upsample + 3x3 conv
+size_t wvae_upsample_conv_packed_bytes(int cout, int cin, wvae_dtype dtype) {
+  if (cout < 1 || cin < 1) return 0;
+  if (dtype == WVAE_BF16) return packed_layout(cout, cin, 1, 4, 4, WVAE_BF16).total;
+  if (dtype == WVAE_F32) return packed_layout(cout, cin, 1, 3, 3, WVAE_F32).total;
+  return 0;
+}
+
+wvae_status wvae_prepack_upsample_conv(const void* w, wvae_dtype w_dtype, const float* bias,
+                                       int cout, int cin, wvae_dtype dtype, void* packed,
+                                       size_t packed_bytes, wvae_stream_t stream) {
+  if (!w || !packed) return WVAE_ERR_INVALID_ARG;
+  if (cout < 1 || cin < 1) return WVAE_ERR_INVALID_ARG;
+  if ((w_dtype != WVAE_BF16 && w_dtype != WVAE_F32) || (dtype != WVAE_BF16 && dtype != WVAE_F32))
+    return WVAE_ERR_UNSUPPORTED;
+  if (!a16(packed)) return WVAE_ERR_ALIGNMENT;
+  if (packed_bytes < wvae_upsample_conv_packed_bytes(cout, cin, dtype)) return WVAE_ERR_WORKSPACE;
+  if (dtype == WVAE_F32)
+    return wvae_prepack_conv(w, w_dtype, bias, cout, cin, 1, 3, 3, WVAE_F32, packed, packed_bytes,
+                             stream);
+  DeviceInfo* d = nullptr;
+  wvae_status st = device_info(&d);
+  if (st != WVAE_OK) return st;
+  const PackedLayout L = packed_layout(cout, cin, 1, 4, 4, WVAE_BF16);
+  float* bias_p = reinterpret_cast<float*>(static_cast<char*>(packed) + L.bias_off);
+  return cuda_status(launch_prepack_phase_bf16(w, w_dtype == WVAE_F32, bias, cout, cin, L.cout_pad,
+                                               L.cin_pad, static_cast<__nv_bfloat16*>(packed),
+                                               bias_p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t wvae_upsample_conv_workspace_bytes(int T, int H, int W, int cin, wvae_dtype dtype) {
-  if (T < 1 || H < 1 || W < 1 || cin < 1) return 0;
+  if (T < 1 || H < 1 || W < 1 || cin < 1 || dtype != WVAE_F32) return 0;
   return round_up_sz(static_cast<size_t>(T) * 4 * H * W * cin * bytes_of(dtype), 256);
 }
 
@@ -485,11 +523,23 @@ wvae_status wvae_upsample_conv(const void* x, void* y, int T, int H, int W, int 
   if (dtype == WVAE_BF16 && (cin % 64 != 0 || !bf16_cout_ok(cout))) return WVAE_ERR_UNSUPPORTED;
   if (dtype == WVAE_F32 && (cin % 4 != 0 || cout % 4 != 0)) return WVAE_ERR_UNSUPPORTED;
   const size_t need = wvae_upsample_conv_workspace_bytes(T, H, W, cin, dtype);
-  if (workspace == nullptr || ws_bytes < need) return WVAE_ERR_WORKSPACE;
+  if (need > 0 && (workspace == nullptr || ws_bytes < need)) return WVAE_ERR_WORKSPACE;
   DeviceInfo* d = nullptr;
   wvae_status st = device_info(&d);
   if (st != WVAE_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == WVAE_BF16) {
+    TcConv c;
+    c.x = x;
+    c.cin_pad = cin;
+    c.packed = packed_w;
+    c.cout = cout;
+    c.T = T; c.H = H; c.W = W;
+    c.phases = 4;
+    c.ep.out = y;
+    c.ep.out_f32 = 0;
+    return run_tc_conv(*d, c, s);
+  }
   st = cuda_status(launch_upsample2x(x, workspace, static_cast<int>(bytes_of(dtype)), T, H, W, cin, s));
   if (st != WVAE_OK) return st;
   return wvae_causal_conv3d(workspace, nullptr, packed_w, T, 2 * H, 2 * W, cin, cout, 1, 3, 3,
@@ -522,7 +572,7 @@ TrunkBuffers trunk_buffers(int T, int H, int W, const int* C) {
     const size_t vs = v0 << (2 * s);
     max_h = std::max(max_h, vs * C[s] * 4);
     max_act = std::max(max_act, vs * C[s] * 2);
-    if (s < 3) max_up = std::max(max_up, (vs << 2) * C[s] * 2);
+    if (s < 3) max_up = std::max(max_up, vs * C[s] * 2);
   }
   b.zcl = take(v0 * kZPad * 2);
   b.h = take(max_h);
@@ -653,10 +703,9 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
         next_norm(&c2.ep.gamma, &c2.ep.beta);
         c2.ep.eps = 1e-12f;
       } else if (stg < 3) {
-        // the stage's output feeds only the upsample conv: write it 2x-upsampled, bf16
+        // the stage's output feeds only the upsample conv (an MMA operand): bf16
         c2.ep.out = up;
         c2.ep.out_f32 = 0;
-        c2.ep.out_upsample2x = 1;
       } else {
         // the last block feeds only norm_out + SiLU + head
         c2.ep.act = act[0];
@@ -667,15 +716,16 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
       if (st != WVAE_OK) return st;
     }
     if (stg < 3) {
-      Hs *= 2;
-      Ws *= 2;
+      // nearest 2x upsample + 3x3 conv as four phase convs on the low-res stage output
       TcConv cu;
       cu.x = up;
       cu.cin_pad = Cs;
       cu.packed = packed[pi++];
       cu.cout = C[stg + 1];
-      cu.KT = 1;
       cu.T = T; cu.H = Hs; cu.W = Ws;
+      cu.phases = 4;
+      Hs *= 2;
+      Ws *= 2;
       cu.ep.out = h;
       cu.ep.out_f32 = 1;
       cu.ep.act = act[0];

@@ -80,13 +80,17 @@ __device__ __forceinline__ Smem carve(uint8_t* raw, const ConvParams& p) {
 }
 
 struct TileCoord {
-  int n_tile, t, th, tw;
+  int n_tile, phase, t, th, tw;
 };
 
+// Tile order: N tile fastest, then upsample phase (the four phases of an M
+// tile read the same input), then M tiles (column, row, frame).
 __device__ __forceinline__ TileCoord decode_tile(const ConvParams& p, int tile) {
   TileCoord c;
   c.n_tile = tile % p.n_tiles;
   int m = tile / p.n_tiles;
+  c.phase = m % p.phases;
+  m /= p.phases;
   c.tw = m % p.tiles_w;
   m /= p.tiles_w;
   c.th = m % p.tiles_h;
@@ -123,13 +127,16 @@ __device__ void producer(const ConvParams& p, const Smem& s) {
         const int kt = tap / kwkh, r = tap - kt * kwkh;
         const int kh = r / p.KW, kw = r - kh * p.KW;
         const int ts = tc.t + kt - (p.KT - 1);
-        const int hs = h0 + kh - (p.KH - 1) / 2;
-        const int ws = w0 + kw - (p.KW - 1) / 2;
+        // phase mode: output (2h+p', 2w+q') reads input rows h + kh + p' - 1
+        const int oh = p.phases == 4 ? (tc.phase >> 1) - 1 : -(p.KH - 1) / 2;
+        const int ow = p.phases == 4 ? (tc.phase & 1) - 1 : -(p.KW - 1) / 2;
+        const int hs = h0 + kh + oh;
+        const int ws = w0 + kw + ow;
         if (ts < 0 && p.has_cache)
           tma_load_4d(a_dst, &p.tmC, bar, cc * kBK, ws, hs, ts + p.KT - 1);
         else
           tma_load_4d(a_dst, &p.tmA, bar, cc * kBK, ws, hs, ts);
-        const int kcoord = tap * p.cin_pad + cc * kBK;
+        const int kcoord = (tc.phase * 4 * (p.phases == 4) + tap) * p.cin_pad + cc * kBK;
         for (int l = 0; l < b_loads; ++l)
           tma_load_2d(b_dst + l * b_box_bytes, &p.tmB, bar, kcoord, tc.n_tile * p.BN + l * 256);
       } else {
@@ -307,30 +314,15 @@ __device__ __forceinline__ void result_chunk(const ConvParams& p, const Smem& s,
 
 template <int NC>
 __device__ __forceinline__ void emit_chunk(const ConvParams& p, const Smem& s, int c0, int n0,
-                                           const TileCoord& tc, int h, int w, size_t vox,
+                                           const TileCoord& tc, int h, int w, size_t ovox,
                                            float rs, float (&v)[NC]) {
   const ConvEpilogue& ep = p.ep;
   if (ep.out != nullptr) {
-    if (!ep.out_upsample2x) {
-      const size_t off = vox * p.cout + n0 + c0;
-      if (ep.out_f32)
-        store_f32<NC>(static_cast<float*>(ep.out) + off, v);
-      else
-        store_bf16<NC>(static_cast<__nv_bfloat16*>(ep.out) + off, v);
-    } else {
-      const int H2 = 2 * p.H, W2 = 2 * p.W;
-#pragma unroll
-      for (int i = 0; i < 2; ++i)
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const size_t v2 = (static_cast<size_t>(tc.t) * H2 + 2 * h + i) * W2 + 2 * w + j;
-          const size_t off = v2 * p.cout + n0 + c0;
-          if (ep.out_f32)
-            store_f32<NC>(static_cast<float*>(ep.out) + off, v);
-          else
-            store_bf16<NC>(static_cast<__nv_bfloat16*>(ep.out) + off, v);
-        }
-    }
+    const size_t off = ovox * p.cout + n0 + c0;
+    if (ep.out_f32)
+      store_f32<NC>(static_cast<float*>(ep.out) + off, v);
+    else
+      store_bf16<NC>(static_cast<__nv_bfloat16*>(ep.out) + off, v);
   }
   if (ep.act != nullptr) {
     float a[NC];
@@ -339,7 +331,7 @@ __device__ __forceinline__ void emit_chunk(const ConvParams& p, const Smem& s, i
       const float sv = v[j] * rs * s.gamma[n0 + c0 + j] + s.beta[n0 + c0 + j];
       a[j] = silu_fast(sv);
     }
-    store_bf16<NC>(ep.act + vox * p.cout + n0 + c0, a);
+    store_bf16<NC>(ep.act + ovox * p.cout + n0 + c0, a);
   }
   if (ep.video != nullptr) {
     const int H2 = 2 * p.H, W2 = 2 * p.W;
@@ -380,7 +372,11 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
     for (int sub = 0; sub < p.S; ++sub) {
       const int h = (tc.th * p.S + sub) * kTileH + hl, w = tc.tw * kTileW + wl;
       const bool valid = h < p.H && w < p.W;
-      const size_t vox = (static_cast<size_t>(tc.t) * p.H + h) * p.W + w;
+      // output voxel: (t, h, w), or (t, 2h + p', 2w + q') of the 2H x 2W output in phase mode
+      const size_t vox = p.phases == 4
+                             ? (static_cast<size_t>(tc.t) * 2 * p.H + 2 * h + (tc.phase >> 1)) *
+                                       (2 * p.W) + 2 * w + (tc.phase & 1)
+                             : (static_cast<size_t>(tc.t) * p.H + h) * p.W + w;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              acc * static_cast<uint32_t>(p.S * p.BN) +
                              static_cast<uint32_t>(sub * p.BN);

@@ -27,9 +27,8 @@ struct ConvEpilogue {
   const float* bias2;       // fp32 [cout_pad] shortcut bias, or null
   const void* residual;     // [T][H][W][cout] or null
   int residual_f32;         // residual dtype: 1 fp32, 0 bf16
-  void* out;                // raw result [T][H][W][cout] (or [T][2H][2W][cout]), or null
+  void* out;                // raw result [T][H][W][cout] ([T][2H][2W][cout] in phase mode), or null
   int out_f32;              // out dtype: 1 fp32, 0 bf16
-  int out_upsample2x;       // 1: write each voxel to its 2x2 block at double resolution
   __nv_bfloat16* act;       // SiLU(norm(result)) bf16 [T][H][W][cout], or null
   const float* gamma;       // fp32 [cout] for act
   const float* beta;        // fp32 [cout] for act
@@ -47,6 +46,7 @@ struct ConvParams {
   int cin_pad, cin2_pad;
   int cout, cout_pad;
   int KT, KH, KW;
+  int phases;        // 4: upsample-conv phase mode (KH = KW = 2, output at (2h+p, 2w+q))
   int has_cache;
   int BN, n_tiles;
   int S;             // MMA sub-tiles per CTA tile; S * BN <= 512 TMEM columns
@@ -84,12 +84,17 @@ cudaError_t launch_norm_silu_f32(const float* x, float* y, const float* gamma, c
 cudaError_t launch_prepack_bf16(const void* w, int w_is_f32, const float* bias, int cout, int cin,
                                 int taps, int cout_pad, int cin_pad, __nv_bfloat16* wp,
                                 float* bias_p, cudaStream_t stream);
+// Upsample-conv weights [cout][cin][1][3][3] -> four 2x2 phase kernels, bf16
+// [cout_pad][16][cin_pad] (see layout.cu).
+cudaError_t launch_prepack_phase_bf16(const void* w, int w_is_f32, const float* bias, int cout,
+                                      int cin, int cout_pad, int cin_pad, __nv_bfloat16* wp,
+                                      float* bias_p, cudaStream_t stream);
 cudaError_t launch_prepack_f32(const void* w, int w_is_f32, const float* bias, int cout, int cin,
                                int taps, float* wp, float* bias_p, cudaStream_t stream);
 // NCDHW [C][T][H][W] bf16 -> channels-last [T][H][W][Cpad] bf16, zero-filled pad channels.
 cudaError_t launch_ncdhw_to_cl_pad(const __nv_bfloat16* x, __nv_bfloat16* y, int C, int Cpad,
                                    int T, int H, int W, cudaStream_t stream);
-// channels-last [T][H][W][C] -> [T][2H][2W][C], nearest.
+// channels-last [T][H][W][C] -> [T][2H][2W][C], nearest (fp32 reference path).
 cudaError_t launch_upsample2x(const void* x, void* y, int elem_bytes, int T, int H, int W, int C,
                               cudaStream_t stream);
 // fp32 [n] -> bf16 [n]

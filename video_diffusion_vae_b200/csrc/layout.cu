@@ -29,6 +29,38 @@ __global__ void prepack_bf16_kernel(const void* w, int is_f32, const float* bias
   }
 }
 
+// Nearest 2x upsample + 3x3 conv as four 2x2 "phase" convs on the low-res
+// input.  Output pixel (2i+p, 2j+q) reads input rows i + r + p - 1 (r = 0, 1)
+// and columns j + c + q - 1 (c = 0, 1); row tap r of phase p combines the
+// 3x3 rows kh in R(p, r): R(0,0) = {0}, R(0,1) = {1,2}, R(1,0) = {0,1},
+// R(1,1) = {2} (and the same for columns).  The combined weights are summed
+// in fp32 and rounded once to bf16.  Packed as [cout_pad][phase*4 + r*2 + c]
+// [cin_pad], phase = 2p + q.
+__device__ __forceinline__ int phase_lo(int p, int r) { return (p == 0) ? (r == 0 ? 0 : 1) : (r == 0 ? 0 : 2); }
+__device__ __forceinline__ int phase_hi(int p, int r) { return (p == 0) ? (r == 0 ? 0 : 2) : (r == 0 ? 1 : 2); }
+
+__global__ void prepack_phase_bf16_kernel(const void* w, int is_f32, const float* bias, int cout,
+                                          int cin, int cout_pad, int cin_pad, __nv_bfloat16* wp,
+                                          float* bias_p) {
+  const long total = static_cast<long>(cout_pad) * 16 * cin_pad;
+  for (long idx = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<long>(gridDim.x) * blockDim.x) {
+    const int i = static_cast<int>(idx % cin_pad);
+    const int tap = static_cast<int>((idx / cin_pad) % 16);
+    const int o = static_cast<int>(idx / (static_cast<long>(cin_pad) * 16));
+    const int phase = tap >> 2, p = phase >> 1, q = phase & 1, r = (tap >> 1) & 1, c = tap & 1;
+    float v = 0.0f;
+    if (o < cout && i < cin) {
+      const long base = (static_cast<long>(o) * cin + i) * 9;
+      for (int kh = phase_lo(p, r); kh <= phase_hi(p, r); ++kh)
+        for (int kw = phase_lo(q, c); kw <= phase_hi(q, c); ++kw)
+          v += load_w(w, is_f32, base + kh * 3 + kw);
+    }
+    wp[idx] = __float2bfloat16_rn(v);
+    if (idx < cout_pad) bias_p[idx] = (bias != nullptr && idx < cout) ? bias[idx] : 0.0f;
+  }
+}
+
 // PyTorch [cout][cin][taps] -> fp32 [taps][cin][cout].
 __global__ void prepack_f32_kernel(const void* w, int is_f32, const float* bias, int cout, int cin,
                                    int taps, float* wp, float* bias_p) {
@@ -90,6 +122,15 @@ cudaError_t launch_prepack_bf16(const void* w, int w_is_f32, const float* bias, 
   const long total = static_cast<long>(cout_pad) * taps * cin_pad;
   prepack_bf16_kernel<<<grid_for(total, 256), 256, 0, stream>>>(w, w_is_f32, bias, cout, cin, taps,
                                                                 cout_pad, cin_pad, wp, bias_p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prepack_phase_bf16(const void* w, int w_is_f32, const float* bias, int cout,
+                                      int cin, int cout_pad, int cin_pad, __nv_bfloat16* wp,
+                                      float* bias_p, cudaStream_t stream) {
+  const long total = static_cast<long>(cout_pad) * 16 * cin_pad;
+  prepack_phase_bf16_kernel<<<grid_for(total, 256), 256, 0, stream>>>(w, w_is_f32, bias, cout, cin,
+                                                                      cout_pad, cin_pad, wp, bias_p);
   return cudaGetLastError();
 }
 
