@@ -21,8 +21,11 @@
 //               tcgen05.mma (M=128, N=BN<=256, K=16) sharing the weight tile,
 //               into TMEM (two accumulators when 2 S BN <= 512, so the
 //               epilogue of tile i overlaps the main loop of tile i+1);
-//   warps 2..5  epilogue: one TMEM lane (= one output voxel per sub-tile) per
-//               thread.
+//   warps 2..9  epilogue, two groups of 4 warps (one warp per TMEM lane
+//               quarter each): one TMEM lane = one output voxel per thread;
+//               with S >= 2 the groups take alternate sub-tiles, with S = 1
+//               each takes half of the channels (the two halves of the RMS
+//               sum meet in shared memory).
 // tcgen05.mma issue runs nearly in step with execution, so every cycle the
 // issuing thread spends waiting on a barrier is a tensor-pipe bubble: S
 // sub-tiles per weight tile put S times more MMA work behind each wait.
@@ -48,6 +51,8 @@ struct Smem {
   uint64_t* tfull;        // [2]
   uint64_t* tempty;       // [2]
   uint64_t* drain;        // [1]
+  uint64_t* ssbar;        // [1] the two epilogue groups' partial RMS sums are written
+  float* ss_part;         // [2 tile parities][2 groups][128 rows]
   uint32_t* tmem_slot;
   int* abort_flag;
   float* bias;            // [512]
@@ -55,7 +60,7 @@ struct Smem {
   float* beta;            // [512]
 };
 
-constexpr uint32_t kCtrlBytes = 512 + 3 * 512 * 4;
+constexpr uint32_t kCtrlBytes = 512 + 3 * 512 * 4 + 2 * 2 * 128 * 4;
 
 __device__ __forceinline__ Smem carve(uint8_t* raw, const ConvParams& p) {
   Smem s;
@@ -71,11 +76,13 @@ __device__ __forceinline__ Smem carve(uint8_t* raw, const ConvParams& p) {
   s.tfull = s.empty + kMaxStages;
   s.tempty = s.tfull + 2;
   s.drain = s.tempty + 2;
-  s.tmem_slot = reinterpret_cast<uint32_t*>(s.drain + 1);
+  s.ssbar = s.drain + 1;
+  s.tmem_slot = reinterpret_cast<uint32_t*>(s.ssbar + 1);
   s.abort_flag = reinterpret_cast<int*>(s.tmem_slot + 1);
   s.bias = reinterpret_cast<float*>(ctrl + 512);
   s.gamma = s.bias + 512;
   s.beta = s.gamma + 512;
+  s.ss_part = s.beta + 512;
   return s;
 }
 
@@ -348,16 +355,55 @@ __device__ __forceinline__ void emit_chunk(const ConvParams& p, const Smem& s, i
   }
 }
 
+// Columns [c_lo, c_hi) of this thread's lane: acc + bias (+ residual), sum of squares.
+__device__ __forceinline__ float lane_sumsq(const ConvParams& p, const Smem& s, uint32_t taddr,
+                                           int c_lo, int c_hi, int n0, bool valid, size_t vox) {
+  float ss = 0.0f;
+  int c0 = c_lo;
+  for (; c0 + 32 <= c_hi; c0 += 32) {
+    float v[32];
+    result_chunk<32>(p, s, taddr, c0, n0, valid, vox, v);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
+  }
+  if (c0 < c_hi) {
+    float v[16];
+    result_chunk<16>(p, s, taddr, c0, n0, valid, vox, v);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) ss = fmaf(v[j], v[j], ss);
+  }
+  return ss;
+}
+
+__device__ __forceinline__ void lane_emit(const ConvParams& p, const Smem& s, uint32_t taddr,
+                                          int c_lo, int c_hi, int n0, bool valid, size_t vox,
+                                          const TileCoord& tc, int h, int w, float rs) {
+  int c0 = c_lo;
+  for (; c0 + 32 <= c_hi; c0 += 32) {
+    float v[32];
+    result_chunk<32>(p, s, taddr, c0, n0, valid, vox, v);
+    if (valid) emit_chunk<32>(p, s, c0, n0, tc, h, w, vox, rs, v);
+  }
+  if (c0 < c_hi) {
+    float v[16];
+    result_chunk<16>(p, s, taddr, c0, n0, valid, vox, v);
+    if (valid) emit_chunk<16>(p, s, c0, n0, tc, h, w, vox, rs, v);
+  }
+}
+
 __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base, int warp,
                          int lane) {
-  const int q = warp & 3;  // TMEM lane quarter this warp may access
+  const int q = warp & 3;           // TMEM lane quarter this warp may access
+  const int grp = (warp - 2) >> 2;  // epilogue group 0 or 1
   const int row = q * 32 + lane;
   const int hl = row / kTileW, wl = row % kTileW;
   const float rootC = sqrtf(static_cast<float>(p.cout));
-  uint32_t ai = 0;
-  for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++ai) {
-    const uint32_t acc = ai % p.num_acc;
-    const uint32_t aph = (ai / p.num_acc) & 1u;
+  const bool split_cols = p.S == 1;
+  const int half = p.BN / 2;
+  uint32_t ti = 0;
+  for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++ti) {
+    const uint32_t acc = ti % p.num_acc;
+    const uint32_t aph = (ti / p.num_acc) & 1u;
     int ok = 0;
     if (lane == 0)
       ok = mbar_wait_bounded(smem_u32(&s.tfull[acc]), aph, s.abort_flag, p.err,
@@ -366,10 +412,11 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
                : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (!ok) break;
+    __syncwarp();  // order the other lanes' reads after lane 0's acquire
     tc_fence_after();
     const TileCoord tc = decode_tile(p, tile);
     const int n0 = tc.n_tile * p.BN;
-    for (int sub = 0; sub < p.S; ++sub) {
+    for (int sub = split_cols ? 0 : grp; sub < p.S; sub += split_cols ? 1 : 2) {
       const int h = (tc.th * p.S + sub) * kTileH + hl, w = tc.tw * kTileW + wl;
       const bool valid = h < p.H && w < p.W;
       // output voxel: (t, h, w), or (t, 2h + p', 2w + q') of the 2H x 2W output in phase mode
@@ -380,35 +427,30 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              acc * static_cast<uint32_t>(p.S * p.BN) +
                              static_cast<uint32_t>(sub * p.BN);
+      const int c_lo = split_cols ? grp * half : 0;
+      const int c_hi = split_cols ? c_lo + half : p.BN;
       float rs = 1.0f;
       if (p.ep.act != nullptr) {
-        float ss = 0.0f;
-        int c0 = 0;
-        for (; c0 + 32 <= p.BN; c0 += 32) {
-          float v[32];
-          result_chunk<32>(p, s, taddr, c0, n0, valid, vox, v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
-        }
-        if (c0 < p.BN) {
-          float v[16];
-          result_chunk<16>(p, s, taddr, c0, n0, valid, vox, v);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) ss = fmaf(v[j], v[j], ss);
+        float ss = lane_sumsq(p, s, taddr, c_lo, c_hi, n0, valid, vox);
+        if (split_cols) {
+          // exchange the two halves' sums through shared memory (bounded wait)
+          float* part = s.ss_part + (ti & 1u) * 256;
+          part[grp * 128 + row] = ss;
+          mbar_arrive(smem_u32(s.ssbar));
+          int got = 0;
+          if (lane == 0)
+            got = mbar_wait_bounded(smem_u32(s.ssbar), ti & 1u, s.abort_flag, p.err,
+                                    DEVERR_TIMEOUT_EPILOGUE)
+                      ? 1
+                      : 0;
+          got = __shfl_sync(0xffffffffu, got, 0);
+          if (!got) return;
+          __syncwarp();
+          ss += part[(grp ^ 1) * 128 + row];
         }
         rs = rootC / fmaxf(sqrtf(ss), p.ep.eps);
       }
-      int c0 = 0;
-      for (; c0 + 32 <= p.BN; c0 += 32) {
-        float v[32];
-        result_chunk<32>(p, s, taddr, c0, n0, valid, vox, v);
-        if (valid) emit_chunk<32>(p, s, c0, n0, tc, h, w, vox, rs, v);
-      }
-      if (c0 < p.BN) {
-        float v[16];
-        result_chunk<16>(p, s, taddr, c0, n0, valid, vox, v);
-        if (valid) emit_chunk<16>(p, s, c0, n0, tc, h, w, vox, rs, v);
-      }
+      lane_emit(p, s, taddr, c_lo, c_hi, n0, valid, vox, tc, h, w, rs);
     }
     tc_fence_before();
     mbar_arrive(smem_u32(&s.tempty[acc]));
@@ -427,9 +469,10 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&s.tfull[i]), 1);
-      mbar_init(smem_u32(&s.tempty[i]), 128);
+      mbar_init(smem_u32(&s.tempty[i]), 256);
     }
     mbar_init(smem_u32(s.drain), 1);
+    mbar_init(smem_u32(s.ssbar), 256);
     *s.abort_flag = 0;
     fence_mbar_init();
   }

@@ -18,7 +18,7 @@ constexpr int kTileH = 8;
 constexpr int kTileW = 16;
 constexpr int kBM = kTileH * kTileW;  // 128
 constexpr int kBK = 64;
-constexpr int kConvThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kConvThreads = 320;     // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue (2 groups)
 constexpr int kMaxStages = 8;
 
 // What the epilogue does with acc + bias (+ residual), per output voxel.
