@@ -41,20 +41,25 @@ L2_FLUSH_BYTES = 512 << 20
 
 
 # ------------------------------------------------------------------ workload
-def trunk_layers(T=T, H=H, W=W, widths=WIDTHS, zc=ZC):
-    """The trunk's launches in order with their dense FLOPs (all taps counted)."""
+def trunk_layers(T=T, H=H, W=W, widths=WIDTHS, zc=ZC, executed=False):
+    """The trunk's launches in order with their dense FLOPs (all taps counted;
+    the upsample convs at output resolution with 9 taps).  executed=True gives
+    the MMA FLOPs the kernels actually issue instead: the upsample convs run as
+    four 2x2 phase convs on the low-res input (16/36 of dense), conv_in runs
+    on 48 channels padded to 64, the head on 12 output channels padded to 16."""
     layers = [("layout", 0.0)]
     v = T * H * W
-    layers.append(("conv_in", 2.0 * v * widths[0] * zc * 27))
+    layers.append(("conv_in", 2.0 * v * widths[0] * (64 if executed else zc) * 27))
     for s, c in enumerate(widths):
         vs = v * 4 ** s
         for b in range(2):
             layers.append((f"s{s}.b{b}.conv1", 2.0 * vs * c * c * 27))
             layers.append((f"s{s}.b{b}.conv2", 2.0 * vs * c * c * 27))
         if s + 1 < len(widths):
-            layers.append((f"s{s}.up", 2.0 * (4 * vs) * widths[s + 1] * c * 9))
+            up = 2.0 * vs * widths[s + 1] * c * 16 if executed else 2.0 * (4 * vs) * widths[s + 1] * c * 9
+            layers.append((f"s{s}.up", up))
     v3 = v * 4 ** (len(widths) - 1)
-    layers.append(("head", 2.0 * v3 * 12 * widths[-1] * 27))
+    layers.append(("head", 2.0 * v3 * (16 if executed else 12) * widths[-1] * 27))
     return layers
 
 
@@ -86,7 +91,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -290,7 +295,7 @@ def profile_case(name: str, launches: int = 3) -> int:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-components", action="store_true")
@@ -365,8 +370,11 @@ def main():
     conv_idx = [j for j, (name, _) in enumerate(layers) if name != "layout"]
     conv_ms = statistics.mean(sum(per_layer[i][j] for j in conv_idx) for i in range(args.steps))
     conv_flops = sum(layers[j][1] for j in conv_idx)
+    exec_layers = trunk_layers(executed=True)
+    conv_flops_exec = sum(exec_layers[j][1] for j in conv_idx)
     conv_launch_ms = conv_ms / len(conv_idx)
     achieved = conv_flops / len(conv_idx) / (conv_launch_ms * 1e-3) / 1e12
+    achieved_exec = conv_flops_exec / len(conv_idx) / (conv_launch_ms * 1e-3) / 1e12
     layer_ms = {layers[j][0]: statistics.mean(per_layer[i][j] for i in range(args.steps)) for j in range(nl)}
 
     # ---- e2e: pinned host latents -> device, decode, video -> pinned host, per step
@@ -419,6 +427,9 @@ def main():
                          "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
                          "frac": achieved / peak_t, "peak_kind": f"{peak_kind} bf16 sustained",
                          "frac_of_burst": achieved / peaks["bf16_tflops"], "frac_of_2250": achieved / 2250.0,
+                         "flops_per_launch": conv_flops / len(conv_idx),
+                         "achieved_executed": achieved_exec,
+                         "frac_executed": achieved_exec / peak_t,
                          "traffic": None, "launch_ms": conv_launch_ms,
                          "conv_share_of_step": conv_ms / statistics.mean(step_ms)},
             "cpu_baseline": cpu,
