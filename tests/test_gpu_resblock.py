@@ -31,8 +31,10 @@ def test_resblock_tiny_config(dtype):
     assert_close(from_cl(y), O.resblock(x, p), dtype, "config 0")
 
 
-@pytest.mark.parametrize("cin,cout", [(256, 256), (256, 128), (128, 64), (64, 128)])
+@pytest.mark.parametrize("cin,cout", [(256, 256), (256, 128), (128, 64), (64, 128), (512, 512)])
 def test_resblock_reduced(cin, cout):
+    """512 -> 512 runs its convs on clusters of two CTAs that split the channels and
+    swap the RMS partial sums over distributed shared memory."""
     x, p = synth.resblock_input(cin=cin, cout=cout, T=3, H=11, W=19, seed=cin + cout)
     blk = B.PackedResBlock(p)
     y = B.resblock(to_cl(x), blk)

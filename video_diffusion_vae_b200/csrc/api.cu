@@ -172,11 +172,16 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   p.KW = a.KW;
   p.phases = a.phases;
   p.has_cache = a.cache != nullptr;
+  // The fused norm needs every output channel of a voxel: one CTA holds them
+  // all (BN = Cout) up to 256; at 512 a cluster of two CTAs splits N and swaps
+  // the partial sums of squares.
   const bool need_all_channels = a.ep.act != nullptr;
+  p.nsplit = 1;
   if (L.cout_pad <= 256) {
     p.BN = L.cout_pad;
   } else if (L.cout_pad == 512) {
-    p.BN = need_all_channels ? 512 : 256;
+    p.BN = 256;
+    if (need_all_channels) p.nsplit = 2;
   } else {
     if (need_all_channels) return WVAE_ERR_UNSUPPORTED;
     p.BN = (L.cout_pad % 256 == 0) ? 256 : (L.cout_pad % 128 == 0 ? 128 : 16);
@@ -189,7 +194,7 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   p.tiles_w = (a.W + kTileW - 1) / kTileW;
   p.tiles_h = (a.H + kTileH * p.S - 1) / (kTileH * p.S);
   p.m_tiles = a.T * p.tiles_h * p.tiles_w;
-  p.num_tiles = p.m_tiles * p.phases * p.n_tiles;
+  p.num_tiles = p.m_tiles * p.phases * (p.nsplit == 2 ? 1 : p.n_tiles);
   p.kblocks_main = a.KT * a.KH * a.KW * (a.cin_pad / kBK);
   p.kblocks = p.kblocks_main + a.cin2_pad / kBK;
   a.ep.bias = reinterpret_cast<const float*>(static_cast<const char*>(a.packed) + L.bias_off);
@@ -210,7 +215,14 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
     if (!encode_act(&p.tmA2, a.x2, a.cin2_pad, a.W, a.H, a.T, box_h)) return WVAE_ERR_CUDA;
     if (!encode_weights(&p.tmB2, a.packed2, a.cin2_pad, L.cout_pad, box_rows)) return WVAE_ERR_CUDA;
   }
-  const int grid = p.num_tiles < d.num_sms ? p.num_tiles : d.num_sms;
+  int grid;
+  if (p.nsplit == 2) {
+    int clusters = conv_tc_max_clusters(p);
+    if (clusters < 1) clusters = d.num_sms / 2;
+    grid = 2 * (p.num_tiles < clusters ? p.num_tiles : clusters);
+  } else {
+    grid = p.num_tiles < d.num_sms ? p.num_tiles : d.num_sms;
+  }
   return cuda_status(launch_conv_tc(p, grid, stream));
 }
 

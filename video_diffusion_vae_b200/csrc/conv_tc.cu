@@ -26,6 +26,10 @@
 //               with S >= 2 the groups take alternate sub-tiles, with S = 1
 //               each takes half of the channels (the two halves of the RMS
 //               sum meet in shared memory).
+// 512 output channels with the next layer's norm fused: a cluster of two CTAs
+// splits N (each runs the S = 2, BN = 256 main loop on its half of the
+// channels for the same M tiles) and the two epilogues exchange each voxel's
+// partial sum of squares through distributed shared memory.
 // tcgen05.mma issue runs nearly in step with execution, so every cycle the
 // issuing thread spends waiting on a barrier is a tensor-pipe bubble: S
 // sub-tiles per weight tile put S times more MMA work behind each wait.
@@ -52,7 +56,9 @@ struct Smem {
   uint64_t* tempty;       // [2]
   uint64_t* drain;        // [1]
   uint64_t* ssbar;        // [1] the two epilogue groups' partial RMS sums are written
+  uint64_t* xbar;         // [2] (per tile parity) the peer CTA's partial sums have arrived
   float* ss_part;         // [2 tile parities][2 groups][128 rows]
+  float* xpart;           // [2 tile parities][256]: partial sums written by the peer CTA
   uint32_t* tmem_slot;
   int* abort_flag;
   float* bias;            // [512]
@@ -60,7 +66,7 @@ struct Smem {
   float* beta;            // [512]
 };
 
-constexpr uint32_t kCtrlBytes = 512 + 3 * 512 * 4 + 2 * 2 * 128 * 4;
+constexpr uint32_t kCtrlBytes = 512 + 3 * 512 * 4 + 2 * 2 * 128 * 4 + 2 * 256 * 4;
 
 __device__ __forceinline__ Smem carve(uint8_t* raw, const ConvParams& p) {
   Smem s;
@@ -77,12 +83,14 @@ __device__ __forceinline__ Smem carve(uint8_t* raw, const ConvParams& p) {
   s.tempty = s.tfull + 2;
   s.drain = s.tempty + 2;
   s.ssbar = s.drain + 1;
-  s.tmem_slot = reinterpret_cast<uint32_t*>(s.ssbar + 1);
+  s.xbar = s.ssbar + 1;
+  s.tmem_slot = reinterpret_cast<uint32_t*>(s.xbar + 2);
   s.abort_flag = reinterpret_cast<int*>(s.tmem_slot + 1);
   s.bias = reinterpret_cast<float*>(ctrl + 512);
   s.gamma = s.bias + 512;
   s.beta = s.gamma + 512;
   s.ss_part = s.beta + 512;
+  s.xpart = s.ss_part + 2 * 2 * 128;
   return s;
 }
 
@@ -92,10 +100,18 @@ struct TileCoord {
 
 // Tile order: N tile fastest, then upsample phase (the four phases of an M
 // tile read the same input), then M tiles (column, row, frame).
-__device__ __forceinline__ TileCoord decode_tile(const ConvParams& p, int tile) {
+// With nsplit = 2 the two CTAs of a cluster take the same tiles and the CTA
+// rank is the N tile.
+__device__ __forceinline__ TileCoord decode_tile(const ConvParams& p, int tile, int crank) {
   TileCoord c;
-  c.n_tile = tile % p.n_tiles;
-  int m = tile / p.n_tiles;
+  int m;
+  if (p.nsplit == 2) {
+    c.n_tile = crank;
+    m = tile;
+  } else {
+    c.n_tile = tile % p.n_tiles;
+    m = tile / p.n_tiles;
+  }
   c.phase = m % p.phases;
   m /= p.phases;
   c.tw = m % p.tiles_w;
@@ -106,7 +122,14 @@ __device__ __forceinline__ TileCoord decode_tile(const ConvParams& p, int tile) 
 }
 
 // ------------------------------------------------------------------ producer
-__device__ void producer(const ConvParams& p, const Smem& s) {
+__device__ __forceinline__ int tile_first(const ConvParams& p) {
+  return p.nsplit == 2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+}
+__device__ __forceinline__ int tile_stride(const ConvParams& p) {
+  return p.nsplit == 2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+}
+
+__device__ void producer(const ConvParams& p, const Smem& s, int crank) {
   const int cchunks = p.cin_pad / kBK;
   const int kwkh = p.KH * p.KW;
   const int b_rows = p.BN > 256 ? 256 : p.BN;
@@ -114,8 +137,8 @@ __device__ void producer(const ConvParams& p, const Smem& s) {
   const uint32_t b_box_bytes = static_cast<uint32_t>(b_rows) * kBK * 2;
   uint32_t it = 0;
   bool aborted = false;
-  for (int tile = blockIdx.x; tile < p.num_tiles && !aborted; tile += gridDim.x) {
-    const TileCoord tc = decode_tile(p, tile);
+  for (int tile = tile_first(p); tile < p.num_tiles && !aborted; tile += tile_stride(p)) {
+    const TileCoord tc = decode_tile(p, tile, crank);
     const int h0 = tc.th * kTileH * p.S, w0 = tc.tw * kTileW;
     for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
       const uint32_t st = it % p.stages;
@@ -190,7 +213,7 @@ __device__ void mma_issuer(const ConvParams& p, const Smem& s, uint32_t tmem_bas
   const uint32_t acc_cols = static_cast<uint32_t>(S) * bn;
   uint32_t st = 0, ph = 0, ai = 0;
   bool aborted = false;
-  for (int tile = blockIdx.x; tile < p.num_tiles && !aborted; tile += gridDim.x, ++ai) {
+  for (int tile = tile_first(p); tile < p.num_tiles && !aborted; tile += tile_stride(p), ++ai) {
     const uint32_t acc = ai % p.num_acc;
     const uint32_t aph = (ai / p.num_acc) & 1u;
     if (!mbar_wait_bounded(smem_u32(&s.tempty[acc]), aph ^ 1u, s.abort_flag, p.err,
@@ -392,7 +415,7 @@ __device__ __forceinline__ void lane_emit(const ConvParams& p, const Smem& s, ui
 }
 
 __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base, int warp,
-                         int lane) {
+                         int lane, int crank) {
   const int q = warp & 3;           // TMEM lane quarter this warp may access
   const int grp = (warp - 2) >> 2;  // epilogue group 0 or 1
   const int row = q * 32 + lane;
@@ -401,7 +424,7 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
   const bool split_cols = p.S == 1;
   const int half = p.BN / 2;
   uint32_t ti = 0;
-  for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++ti) {
+  for (int tile = tile_first(p); tile < p.num_tiles; tile += tile_stride(p), ++ti) {
     const uint32_t acc = ti % p.num_acc;
     const uint32_t aph = (ti / p.num_acc) & 1u;
     int ok = 0;
@@ -414,7 +437,7 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
     if (!ok) break;
     __syncwarp();  // order the other lanes' reads after lane 0's acquire
     tc_fence_after();
-    const TileCoord tc = decode_tile(p, tile);
+    const TileCoord tc = decode_tile(p, tile, crank);
     const int n0 = tc.n_tile * p.BN;
     for (int sub = split_cols ? 0 : grp; sub < p.S; sub += split_cols ? 1 : 2) {
       const int h = (tc.th * p.S + sub) * kTileH + hl, w = tc.tw * kTileW + wl;
@@ -432,7 +455,23 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
       float rs = 1.0f;
       if (p.ep.act != nullptr) {
         float ss = lane_sumsq(p, s, taddr, c_lo, c_hi, n0, valid, vox);
-        if (split_cols) {
+        if (p.nsplit == 2) {
+          // the other half of the channels is in the peer CTA: swap partial sums
+          const int slot = (ti & 1u) * 256 + sub * 128 + row;
+          const uint32_t peer = static_cast<uint32_t>(crank ^ 1);
+          st_shared_cluster_f32(mapa_shared(smem_u32(&s.xpart[slot]), peer), ss);
+          mbar_arrive_cluster(mapa_shared(smem_u32(&s.xbar[ti & 1u]), peer));
+          int got = 0;
+          if (lane == 0)
+            got = mbar_wait_cluster_bounded(smem_u32(&s.xbar[ti & 1u]), (ti >> 1) & 1u,
+                                            s.abort_flag, p.err, DEVERR_TIMEOUT_EPILOGUE)
+                      ? 1
+                      : 0;
+          got = __shfl_sync(0xffffffffu, got, 0);
+          if (!got) return;
+          __syncwarp();
+          ss += s.xpart[slot];
+        } else if (split_cols) {
           // exchange the two halves' sums through shared memory (bounded wait)
           float* part = s.ss_part + (ti & 1u) * 256;
           part[grp * 128 + row] = ss;
@@ -473,6 +512,8 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
     }
     mbar_init(smem_u32(s.drain), 1);
     mbar_init(smem_u32(s.ssbar), 256);
+    mbar_init(smem_u32(&s.xbar[0]), 256);  // 256 epilogue threads of the peer CTA
+    mbar_init(smem_u32(&s.xbar[1]), 256);
     *s.abort_flag = 0;
     fence_mbar_init();
   }
@@ -495,11 +536,14 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
   }
   tc_fence_before();
   __syncthreads();
+  // With a CTA pair, both CTAs' barriers exist before either writes to the other.
+  if (p.nsplit == 2) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *s.tmem_slot;
+  const int crank = p.nsplit == 2 ? static_cast<int>(cluster_ctarank()) : 0;
 
   if (warp == 0) {
-    if (lane == 0) producer(p, s);
+    if (lane == 0) producer(p, s, crank);
   } else if (warp == 1) {
     if (lane == 0) {
       if (p.BN > 256)
@@ -512,11 +556,13 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
         mma_issuer<4, 1>(p, s, tmem_base);
     }
   } else {
-    epilogue(p, s, tmem_base, warp, lane);
+    epilogue(p, s, tmem_base, warp, lane, crank);
   }
 
   tc_fence_before();
   __syncthreads();
+  // Neither CTA of a pair leaves while the other may still write into it.
+  if (p.nsplit == 2) cluster_sync_all();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -538,15 +584,58 @@ int conv_tc_stages_for(int BN, int S) {
   return st;
 }
 
-cudaError_t launch_conv_tc(const ConvParams& p, int grid, cudaStream_t stream) {
+namespace {
+size_t launch_smem(const ConvParams& p) {
   // Every CTA allocates all 512 TMEM columns, so exactly one may live on an SM:
   // ask for more than half of the SM's shared memory even when the ring is small.
   size_t smem = conv_tc_smem_bytes(p.BN, p.S, p.stages);
   if (smem < 120 * 1024) smem = 120 * 1024;
+  return smem;
+}
+
+cudaLaunchConfig_t launch_config(const ConvParams& p, int grid, size_t smem, cudaStream_t stream,
+                                 cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kConvThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.nsplit == 2 ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+}  // namespace
+
+int conv_tc_max_clusters(const ConvParams& p) {
+  const size_t smem = launch_smem(p);
+  if (cudaFuncSetAttribute(conv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = launch_config(p, 2, smem, nullptr, attr);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, conv_tc_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+cudaError_t launch_conv_tc(const ConvParams& p, int grid, cudaStream_t stream) {
+  const size_t smem = launch_smem(p);
   cudaError_t e = cudaFuncSetAttribute(conv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  conv_tc_kernel<<<grid, kConvThreads, smem, stream>>>(p);
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = launch_config(p, grid, smem, stream, attr);
+  e = cudaLaunchKernelEx(&cfg, conv_tc_kernel, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

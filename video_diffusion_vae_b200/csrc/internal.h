@@ -47,6 +47,8 @@ struct ConvParams {
   int cout, cout_pad;
   int KT, KH, KW;
   int phases;        // 4: upsample-conv phase mode (KH = KW = 2, output at (2h+p, 2w+q))
+  int nsplit;        // 2: a cluster of 2 CTAs splits N (rank = N tile) and exchanges the
+                     //    RMS partial sums over distributed shared memory
   int has_cache;
   int BN, n_tiles;
   int S;             // MMA sub-tiles per CTA tile; S * BN <= 512 TMEM columns
@@ -59,6 +61,8 @@ struct ConvParams {
 
 size_t conv_tc_smem_bytes(int BN, int S, int stages);
 int conv_tc_stages_for(int BN, int S);
+// Clusters of 2 that fit on the device at once (nsplit = 2 launches), 0 on error.
+int conv_tc_max_clusters(const ConvParams& p);
 cudaError_t launch_conv_tc(const ConvParams& p, int grid, cudaStream_t stream);
 
 // ------------------------------------------------------------ fp32 direct conv
