@@ -19,6 +19,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import hashlib
 import json
 import os
 import statistics
@@ -70,6 +71,38 @@ def load_peaks():
         return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
     except Exception:
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------ DRAM traffic
+KERNEL_SOURCES = ("conv_tc.cu", "api.cu", "internal.h", "ptx.cuh")
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "conv_tc_trunk_dram_4x44x78.md")
+
+
+def conv_source_hash() -> str:
+    """Hash of the sources that decide what the conv kernel reads and writes."""
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "video_diffusion_vae_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def conv_traffic():
+    """Mean DRAM bytes (read + write) per conv launch of a trunk step, from the
+    committed ncu capture, or None when that capture was taken on other kernel
+    sources (its `source_hash` line differs) or is missing."""
+    try:
+        kv = {}
+        with open(TRAFFIC_PROFILE) as fh:
+            for line in fh:
+                if line.startswith("- ") and ":" in line:
+                    k, v = line[2:].split(":", 1)
+                    kv[k.strip()] = v.strip().strip("`")
+        if kv.get("source_hash") != conv_source_hash():
+            return None
+        return float(kv["dram_bytes_per_conv_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 # ------------------------------------------------------------------- clocks
@@ -256,7 +289,8 @@ def profile_case(name: str, launches: int = 3) -> int:
     """Run one kernel workload `launches` times (for an ncu capture; no JSON line).
     conv512: causal conv 512->512 on [4,88,156]; norm512 / norm256: norm-SiLU on
     [512,4,88,156] / [256,4,176,312]; res256: res block 256->256 on [4,176,312];
-    trunk: one trunk decode."""
+    res128: res block 128->128 on [4,352,624] (the last stage's shape); trunk:
+    one trunk decode."""
     import torch
     from video_diffusion_vae_b200 import binding as B
     from video_diffusion_vae_b200 import synth
@@ -274,6 +308,11 @@ def profile_case(name: str, launches: int = 3) -> int:
         fn = lambda: B.norm_silu(xd, gd, bd)  # noqa: E731
     elif name == "res256":
         x, p = synth.resblock_input()
+        blk = B.PackedResBlock(p)
+        xd = x.permute(1, 2, 3, 0).contiguous().cuda().bfloat16()
+        fn = lambda: B.resblock(xd, blk)  # noqa: E731
+    elif name == "res128":
+        x, p = synth.resblock_input(cin=128, cout=128, T=4, H=352, W=624)
         blk = B.PackedResBlock(p)
         xd = x.permute(1, 2, 3, 0).contiguous().cuda().bfloat16()
         fn = lambda: B.resblock(xd, blk)  # noqa: E731
@@ -302,7 +341,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", default=None,
                     help="run one kernel workload for an ncu capture (conv512, norm512, norm256, "
-                         "res256, trunk) and exit")
+                         "res256, res128, trunk) and exit")
     args = ap.parse_args()
     if args.profile_case:
         return profile_case(args.profile_case)
@@ -430,7 +469,8 @@ def main():
                          "flops_per_launch": conv_flops / len(conv_idx),
                          "achieved_executed": achieved_exec,
                          "frac_executed": achieved_exec / peak_t,
-                         "traffic": None, "launch_ms": conv_launch_ms,
+                         "traffic": conv_traffic(), "traffic_unit": "bytes per launch (mean of the 21)",
+                         "launch_ms": conv_launch_ms,
                          "conv_share_of_step": conv_ms / statistics.mean(step_ms)},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": zh.numel() * 2,

@@ -39,12 +39,13 @@ def test_conv_kernel_sizes_two_chunks(k):
     assert_close(from_cl(y), O.causal_conv3d(x, w, b), torch.bfloat16, f"k={k}")
 
 
-@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_conv_with_residual_norm_and_cache(dtype):
+@pytest.mark.parametrize("dtype,cout", [(torch.bfloat16, 64), (torch.float32, 64), (torch.bfloat16, 128)])
+def test_conv_with_residual_norm_and_cache(dtype, cout):
+    """cout = 64 runs the row-halo main loop (one A load per (kt, kw) window)."""
     bf = dtype == torch.bfloat16
-    x, w, b = synth.conv_input(cin=64, cout=64, T=3, H=10, W=18, seed=11, bf16=bf)
+    x, w, b = synth.conv_input(cin=64, cout=cout, T=3, H=10, W=18, seed=11, bf16=bf)
     g = torch.Generator().manual_seed(12)
-    res = torch.randn(64, 3, 10, 18, generator=g)
+    res = torch.randn(cout, 3, 10, 18, generator=g)
     res = res.to(torch.bfloat16).float() if bf else res
     gamma = 1 + 0.3 * torch.randn(64, generator=g)
     beta = 0.3 * torch.randn(64, generator=g)
@@ -86,5 +87,26 @@ def test_conv_full_size_sampled():
     got = np.stack([yc[t, h, ww].double().numpy() for (t, h, ww) in pts], 1)
     ref = np.stack([O.causal_conv3d_at(x, w, b, t, h, ww) for (t, h, ww) in pts], 1)
     assert_close(got, ref, torch.bfloat16, "config 2 sampled")
+    assert torch.isfinite(yc).all()
+    assert B.device_error() == 0
+
+
+def test_conv_wide_tiles_sampled():
+    """128 -> 128 on [128, 13, 40, 60]: with 148 SMs, CTA tiles of 8 x 32 voxels
+    (130 tiles; each MMA sub-tile is 4 rows x 32 columns) need fewer waves than
+    16 x 16 tiles (156), so this layer takes the wide shape, ragged in W."""
+    T, H, W = 13, 40, 60
+    x, w, b = synth.conv_input(cin=128, cout=128, T=T, H=H, W=W, seed=5)
+    pk = B.prepack_conv(w.cuda().bfloat16(), b.cuda())
+    y = B.causal_conv3d(to_cl(x), pk)
+    torch.cuda.synchronize()
+    yc = y.float().cpu()
+    pts = set(sample_voxels(T, H, W, 40, seed=4))
+    # both sub-tiles of a tile (rows 3 | 4), tile seams, the ragged last tile
+    pts |= {(0, 3, 31), (0, 4, 0), (1, 7, 31), (2, 8, 32), (12, 35, 47), (12, 36, 48), (6, 20, 59)}
+    pts = sorted(pts)
+    got = np.stack([yc[t, h, ww].double().numpy() for (t, h, ww) in pts], 1)
+    ref = np.stack([O.causal_conv3d_at(x, w, b, t, h, ww) for (t, h, ww) in pts], 1)
+    assert_close(got, ref, torch.bfloat16, "wide tiles sampled")
     assert torch.isfinite(yc).all()
     assert B.device_error() == 0

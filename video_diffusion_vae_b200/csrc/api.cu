@@ -108,12 +108,12 @@ PackedLayout packed_layout(int cout, int cin, int kt, int kh, int kw, wvae_dtype
 }
 
 // ------------------------------------------------------------ TMA descriptors
-bool encode_act(CUtensorMap* m, const void* base, int C, int W, int H, int T, int box_h) {
+bool encode_act(CUtensorMap* m, const void* base, int C, int W, int H, int T, int box_w, int box_h) {
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(W),
                         static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(C) * 2, static_cast<cuuint64_t>(C) * 2 * W,
                            static_cast<cuuint64_t>(C) * 2 * W * H};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(kTileW),
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_w),
                        static_cast<cuuint32_t>(box_h), 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
@@ -189,13 +189,35 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   p.n_tiles = L.cout_pad / p.BN;
   // Sub-tiles per CTA tile: S M=128 MMAs share each weight tile (see conv_tc.cu).
   p.S = p.BN >= 512 ? 1 : (p.BN >= 128 ? 2 : 4);
+  // Narrow layers (the head) are bound by refilling A once per tap: load each
+  // (kt, kw) window once with its row halo and run the KH row taps from it.
+  p.rowhalo = (p.BN <= 64 && a.KH == 3 && a.phases == 1 && a.cin2_pad == 0 && p.nsplit == 1) ? 1 : 0;
+  if (p.rowhalo) p.S = 2;
   p.num_acc = 2 * p.S * p.BN <= 512 ? 2 : 1;
-  p.stages = conv_tc_stages_for(p.BN, p.S);
-  p.tiles_w = (a.W + kTileW - 1) / kTileW;
-  p.tiles_h = (a.H + kTileH * p.S - 1) / (kTileH * p.S);
+  // Tile shape: 128 S voxels as tile_rows x tile_cols, tile_cols in {16, 32,
+  // 64}; the narrowest shape among those needing the fewest waves of tiles over
+  // the CTAs (or CTA pairs) that run at once.
+  const int slots = p.nsplit == 2 ? d.num_sms / 2 : d.num_sms;
+  const int per_m = p.phases * (p.nsplit == 2 ? 1 : p.n_tiles);
+  auto waves = [&](int rows, int cols) {
+    const long tiles = static_cast<long>(a.T) * ((a.H + rows - 1) / rows) * ((a.W + cols - 1) / cols) * per_m;
+    return (tiles + slots - 1) / slots;
+  };
+  p.tile_cols = kTileW;
+  p.tile_rows = kBM * p.S / kTileW;
+  for (int cols = 2 * kTileW; cols <= 64 && kBM * p.S / cols >= kTileH; cols *= 2) {
+    if (waves(kBM * p.S / cols, cols) < waves(p.tile_rows, p.tile_cols)) {
+      p.tile_cols = cols;
+      p.tile_rows = kBM * p.S / cols;
+    }
+  }
+  p.tile_cols_log2 = p.tile_cols == 16 ? 4 : (p.tile_cols == 32 ? 5 : 6);
+  p.stages = conv_tc_stages_for(p);
+  p.tiles_w = (a.W + p.tile_cols - 1) / p.tile_cols;
+  p.tiles_h = (a.H + p.tile_rows - 1) / p.tile_rows;
   p.m_tiles = a.T * p.tiles_h * p.tiles_w;
-  p.num_tiles = p.m_tiles * p.phases * (p.nsplit == 2 ? 1 : p.n_tiles);
-  p.kblocks_main = a.KT * a.KH * a.KW * (a.cin_pad / kBK);
+  p.num_tiles = p.m_tiles * per_m;
+  p.kblocks_main = (p.rowhalo ? a.KT * a.KW : a.KT * a.KH * a.KW) * (a.cin_pad / kBK);
   p.kblocks = p.kblocks_main + a.cin2_pad / kBK;
   a.ep.bias = reinterpret_cast<const float*>(static_cast<const char*>(a.packed) + L.bias_off);
   if (a.packed2 != nullptr) {
@@ -205,14 +227,16 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   p.ep = a.ep;
   p.err = d.err;
   const int box_rows = p.BN > 256 ? 256 : p.BN;
-  const int box_h = kTileH * p.S;
-  if (!encode_act(&p.tmA, a.x, a.cin_pad, a.W, a.H, a.T, box_h)) return WVAE_ERR_CUDA;
+  const int a_rows = p.rowhalo ? p.tile_rows + a.KH - 1 : p.tile_rows;
+  if (!encode_act(&p.tmA, a.x, a.cin_pad, a.W, a.H, a.T, p.tile_cols, a_rows))
+    return WVAE_ERR_CUDA;
   if (!encode_weights(&p.tmB, a.packed, L.taps * a.cin_pad, L.cout_pad, box_rows))
     return WVAE_ERR_CUDA;
-  if (a.cache != nullptr && !encode_act(&p.tmC, a.cache, a.cin_pad, a.W, a.H, a.KT - 1, box_h))
+  if (a.cache != nullptr && !encode_act(&p.tmC, a.cache, a.cin_pad, a.W, a.H, a.KT - 1, p.tile_cols,
+                                        a_rows))
     return WVAE_ERR_CUDA;
   if (a.cin2_pad > 0) {
-    if (!encode_act(&p.tmA2, a.x2, a.cin2_pad, a.W, a.H, a.T, box_h)) return WVAE_ERR_CUDA;
+    if (!encode_act(&p.tmA2, a.x2, a.cin2_pad, a.W, a.H, a.T, p.tile_cols, p.tile_rows)) return WVAE_ERR_CUDA;
     if (!encode_weights(&p.tmB2, a.packed2, a.cin2_pad, L.cout_pad, box_rows)) return WVAE_ERR_CUDA;
   }
   int grid;

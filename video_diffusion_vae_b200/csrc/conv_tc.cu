@@ -13,10 +13,12 @@
 // operands, fp32 accumulation; temporal caching: TensorRT-LLM issue #19309,
 // "Feature, motivation and proposed scope".)
 //
-// One CTA per SM, persistent over output tiles of 8S rows x 16 columns of one
-// frame (S MMA sub-tiles of 128 voxels) x BN output channels.  Warp roles:
-//   warp 0      TMA producer: A box {64 ch, 16 w, 8S h, 1 t} + B box {64, BN}
-//               per K block into a ring of `stages` shared-memory stages;
+// One CTA per SM, persistent over output tiles of tile_rows x tile_cols voxels
+// of one frame (128 S voxels: S MMA sub-tiles of 128 consecutive voxels in
+// row-major order; the shape is chosen per layer to balance the waves) x BN
+// output channels.  Warp roles:
+//   warp 0      TMA producer: A box {64 ch, tile_cols w, tile_rows h, 1 t} +
+//               B box {64, BN} per K block into a ring of `stages` stages;
 //   warp 1      MMA issuer: per K block, 4 K steps x S sub-tiles of
 //               tcgen05.mma (M=128, N=BN<=256, K=16) sharing the weight tile,
 //               into TMEM (two accumulators when 2 S BN <= 512, so the
@@ -50,6 +52,7 @@ struct Smem {
   uint8_t* stages;        // stage s at stages + s * stage_bytes, 1024-aligned
   uint32_t stage_bytes;
   uint32_t a_bytes;
+  uint32_t tx_bytes;      // bytes the TMA loads of one main-loop stage deliver
   uint64_t* full;         // [kMaxStages]
   uint64_t* empty;        // [kMaxStages]
   uint64_t* tfull;        // [2]
@@ -73,8 +76,11 @@ __device__ __forceinline__ Smem carve(uint8_t* raw, const ConvParams& p) {
   uint32_t base = smem_u32(raw);
   uint32_t pad = (1024u - (base & 1023u)) & 1023u;
   uint8_t* al = raw + pad;
-  s.a_bytes = static_cast<uint32_t>(kBM) * p.S * kBK * 2;
-  s.stage_bytes = s.a_bytes + static_cast<uint32_t>(p.BN) * kBK * 2;
+  s.a_bytes = conv_tc_a_bytes(p);
+  s.stage_bytes = s.a_bytes + conv_tc_b_bytes(p);
+  s.tx_bytes = (p.rowhalo ? static_cast<uint32_t>(p.tile_rows + p.KH - 1) : static_cast<uint32_t>(p.tile_rows)) *
+                   static_cast<uint32_t>(p.tile_cols) * 128u +
+               conv_tc_b_bytes(p);
   s.stages = al;
   uint8_t* ctrl = al + p.stages * s.stage_bytes;
   s.full = reinterpret_cast<uint64_t*>(ctrl);
@@ -139,7 +145,7 @@ __device__ void producer(const ConvParams& p, const Smem& s, int crank) {
   bool aborted = false;
   for (int tile = tile_first(p); tile < p.num_tiles && !aborted; tile += tile_stride(p)) {
     const TileCoord tc = decode_tile(p, tile, crank);
-    const int h0 = tc.th * kTileH * p.S, w0 = tc.tw * kTileW;
+    const int h0 = tc.th * p.tile_rows, w0 = tc.tw * p.tile_cols;
     for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
       const uint32_t st = it % p.stages;
       const uint32_t ph = (it / p.stages) & 1u;
@@ -151,7 +157,26 @@ __device__ void producer(const ConvParams& p, const Smem& s, int crank) {
       const uint32_t bar = smem_u32(&s.full[st]);
       const uint32_t a_dst = smem_u32(s.stages + st * s.stage_bytes);
       const uint32_t b_dst = a_dst + s.a_bytes;
-      mbar_arrive_expect_tx(bar, s.stage_bytes);
+      if (p.rowhalo && kb < p.kblocks_main) {
+        // (kt, kw, channel chunk): rows h0 - (KH-1)/2 .. h0 + tile_rows + KH/2 once,
+        // the KH row taps' weight tiles side by side
+        mbar_arrive_expect_tx(bar, s.tx_bytes);
+        const int tap2 = kb / cchunks, cc = kb - tap2 * cchunks;
+        const int kt = tap2 / p.KW, kw = tap2 - kt * p.KW;
+        const int ts = tc.t + kt - (p.KT - 1);
+        const int hs = h0 - (p.KH - 1) / 2, ws = w0 + kw - (p.KW - 1) / 2;
+        if (ts < 0 && p.has_cache)
+          tma_load_4d(a_dst, &p.tmC, bar, cc * kBK, ws, hs, ts + p.KT - 1);
+        else
+          tma_load_4d(a_dst, &p.tmA, bar, cc * kBK, ws, hs, ts);
+        for (int kh = 0; kh < p.KH; ++kh) {
+          const int tap = (kt * p.KH + kh) * p.KW + kw;
+          tma_load_2d(b_dst + kh * static_cast<uint32_t>(p.BN) * 128u, &p.tmB, bar,
+                      tap * p.cin_pad + cc * kBK, tc.n_tile * p.BN);
+        }
+        continue;
+      }
+      mbar_arrive_expect_tx(bar, s.tx_bytes);
       if (kb < p.kblocks_main) {
         const int tap = kb / cchunks, cc = kb - tap * cchunks;
         const int kt = tap / kwkh, r = tap - kt * kwkh;
@@ -196,8 +221,10 @@ __device__ __noinline__ bool mma_wait_slow(uint32_t bar, uint32_t parity, volati
 
 // S sub-tiles and HALVES weight halves are compile-time so the issue loop is
 // fully unrolled: the thread must hand the next MMA to the tensor core as soon
-// as it can take it.
-template <int S, int HALVES>
+// as it can take it.  KHT > 1 (row-halo mode): each K step runs the KHT row taps, the A operand
+// shifted down by one tile row (tile_cols voxels, whole 8-row swizzle atoms)
+// and the B operand moved to that tap's weight tile.
+template <int S, int HALVES, int KHT>
 __device__ void mma_issuer(const ConvParams& p, const Smem& s, uint32_t tmem_base) {
   const int n_inst = p.BN > 256 ? 256 : p.BN;
   const uint32_t idesc = umma_idesc_bf16(kBM, n_inst);
@@ -208,6 +235,8 @@ __device__ void mma_issuer(const ConvParams& p, const Smem& s, uint32_t tmem_bas
   const uint64_t bdesc0 = umma_desc_sw128(smem_u32(s.stages) + s.a_bytes);
   const uint32_t stage_step = s.stage_bytes >> 4;
   const uint32_t sub_step = (static_cast<uint32_t>(kBM) * 128u) >> 4;
+  const uint32_t kh_step_a = static_cast<uint32_t>(p.tile_cols) * 8u;  // tile_cols * 128 B / 16
+  const uint32_t kh_step_b = static_cast<uint32_t>(p.BN) * 8u;
   const uint32_t full0 = smem_u32(&s.full[0]), empty0 = smem_u32(&s.empty[0]);
   const uint32_t bn = static_cast<uint32_t>(p.BN);
   const uint32_t acc_cols = static_cast<uint32_t>(S) * bn;
@@ -234,13 +263,17 @@ __device__ void mma_issuer(const ConvParams& p, const Smem& s, uint32_t tmem_bas
       const uint64_t b_st = bdesc0 + st * stage_step;
 #pragma unroll
       for (int k = 0; k < kBK / 16; ++k) {
-        const uint32_t accumulate = (kb | k) != 0 ? 1u : 0u;
 #pragma unroll
-        for (int sub = 0; sub < S; ++sub) {
-          const uint64_t a_k = a_st + sub * sub_step + 2u * k;
-          const uint32_t d_sub = d_tmem + static_cast<uint32_t>(sub) * bn;
-          umma_bf16(d_sub, a_k, b_st + 2u * k, idesc, accumulate);
-          if (HALVES == 2) umma_bf16(d_sub + 256u, a_k, b_st + 2048u + 2u * k, idesc, accumulate);
+        for (int kh = 0; kh < KHT; ++kh) {
+          const uint32_t accumulate = (kb | k | kh) != 0 ? 1u : 0u;
+          const uint64_t b_k = b_st + kh * kh_step_b + 2u * k;
+#pragma unroll
+          for (int sub = 0; sub < S; ++sub) {
+            const uint64_t a_k = a_st + sub * sub_step + kh * kh_step_a + 2u * k;
+            const uint32_t d_sub = d_tmem + static_cast<uint32_t>(sub) * bn;
+            umma_bf16(d_sub, a_k, b_k, idesc, accumulate);
+            if (HALVES == 2) umma_bf16(d_sub + 256u, a_k, b_k + 2048u, idesc, accumulate);
+          }
         }
       }
       umma_commit(empty0 + st * 8u);
@@ -343,9 +376,8 @@ __device__ __forceinline__ void result_chunk(const ConvParams& p, const Smem& s,
 }
 
 template <int NC>
-__device__ __forceinline__ void emit_chunk(const ConvParams& p, const Smem& s, int c0, int n0,
-                                           const TileCoord& tc, int h, int w, size_t ovox,
-                                           float rs, float (&v)[NC]) {
+__device__ __forceinline__ void store_raw(const ConvParams& p, int c0, int n0, size_t ovox,
+                                          const float (&v)[NC]) {
   const ConvEpilogue& ep = p.ep;
   if (ep.out != nullptr) {
     const size_t off = ovox * p.cout + n0 + c0;
@@ -354,15 +386,26 @@ __device__ __forceinline__ void emit_chunk(const ConvParams& p, const Smem& s, i
     else
       store_bf16<NC>(static_cast<__nv_bfloat16*>(ep.out) + off, v);
   }
-  if (ep.act != nullptr) {
-    float a[NC];
+}
+
+template <int NC>
+__device__ __forceinline__ void store_act(const ConvParams& p, const Smem& s, int c0, int n0,
+                                          size_t ovox, float rs, const float (&v)[NC]) {
+  float a[NC];
 #pragma unroll
-    for (int j = 0; j < NC; ++j) {
-      const float sv = v[j] * rs * s.gamma[n0 + c0 + j] + s.beta[n0 + c0 + j];
-      a[j] = silu_fast(sv);
-    }
-    store_bf16<NC>(ep.act + ovox * p.cout + n0 + c0, a);
+  for (int j = 0; j < NC; ++j) {
+    a[j] = silu_half(v[j] * rs * s.gamma[n0 + c0 + j] + s.beta[n0 + c0 + j]);
   }
+  store_bf16<NC>(p.ep.act + ovox * p.cout + n0 + c0, a);
+}
+
+// Outputs that need no RMS statistic: the raw result and the video.
+template <int NC>
+__device__ __forceinline__ void emit_chunk(const ConvParams& p, int c0, int n0,
+                                           const TileCoord& tc, int h, int w, size_t ovox,
+                                           const float (&v)[NC]) {
+  const ConvEpilogue& ep = p.ep;
+  store_raw<NC>(p, c0, n0, ovox, v);
   if (ep.video != nullptr) {
     const int H2 = 2 * p.H, W2 = 2 * p.W;
 #pragma unroll
@@ -378,39 +421,72 @@ __device__ __forceinline__ void emit_chunk(const ConvParams& p, const Smem& s, i
   }
 }
 
-// Columns [c_lo, c_hi) of this thread's lane: acc + bias (+ residual), sum of squares.
-__device__ __forceinline__ float lane_sumsq(const ConvParams& p, const Smem& s, uint32_t taddr,
+template <int NC>
+__device__ __forceinline__ void tmem_store_chunk(uint32_t taddr, const float (&v)[NC]) {
+  uint32_t r[NC];
+#pragma unroll
+  for (int j = 0; j < NC; ++j) r[j] = __float_as_uint(v[j]);
+  if constexpr (NC == 32)
+    tmem_st32(taddr, r);
+  else
+    tmem_st16(taddr, r);
+}
+
+// First pass over columns [c_lo, c_hi) of this thread's lane when the next
+// layer's norm is fused: h = acc + bias (+ residual) goes out raw (if asked),
+// back into the lane (so the second pass reads neither the residual nor the
+// bias again), and into the returned sum of squares.
+template <int NC>
+__device__ __forceinline__ void pass1_chunk(const ConvParams& p, const Smem& s, uint32_t taddr,
+                                            int c0, int n0, bool valid, size_t vox, float& ss) {
+  float v[NC];
+  result_chunk<NC>(p, s, taddr, c0, n0, valid, vox, v);
+#pragma unroll
+  for (int j = 0; j < NC; ++j) ss = fmaf(v[j], v[j], ss);
+  if (valid) store_raw<NC>(p, c0, n0, vox, v);
+  tmem_store_chunk<NC>(taddr + c0, v);
+}
+__device__ __forceinline__ float lane_pass1(const ConvParams& p, const Smem& s, uint32_t taddr,
                                            int c_lo, int c_hi, int n0, bool valid, size_t vox) {
   float ss = 0.0f;
   int c0 = c_lo;
-  for (; c0 + 32 <= c_hi; c0 += 32) {
-    float v[32];
-    result_chunk<32>(p, s, taddr, c0, n0, valid, vox, v);
-#pragma unroll
-    for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
-  }
-  if (c0 < c_hi) {
-    float v[16];
-    result_chunk<16>(p, s, taddr, c0, n0, valid, vox, v);
-#pragma unroll
-    for (int j = 0; j < 16; ++j) ss = fmaf(v[j], v[j], ss);
-  }
+  for (; c0 + 32 <= c_hi; c0 += 32) pass1_chunk<32>(p, s, taddr, c0, n0, valid, vox, ss);
+  if (c0 < c_hi) pass1_chunk<16>(p, s, taddr, c0, n0, valid, vox, ss);
+  tmem_wait_st();
   return ss;
 }
 
+// Second pass: the next layer's activation SiLU(h r gamma + beta) from h in the lane.
+__device__ __forceinline__ void lane_pass2(const ConvParams& p, const Smem& s, uint32_t taddr,
+                                          int c_lo, int c_hi, int n0, bool valid, size_t vox,
+                                          float rs) {
+  int c0 = c_lo;
+  for (; c0 + 32 <= c_hi; c0 += 32) {
+    float v[32];
+    tmem_load_chunk<32>(taddr + c0, v);
+    if (valid) store_act<32>(p, s, c0, n0, vox, rs, v);
+  }
+  if (c0 < c_hi) {
+    float v[16];
+    tmem_load_chunk<16>(taddr + c0, v);
+    if (valid) store_act<16>(p, s, c0, n0, vox, rs, v);
+  }
+}
+
+// Single pass when no norm is fused: raw result and / or video.
 __device__ __forceinline__ void lane_emit(const ConvParams& p, const Smem& s, uint32_t taddr,
                                           int c_lo, int c_hi, int n0, bool valid, size_t vox,
-                                          const TileCoord& tc, int h, int w, float rs) {
+                                          const TileCoord& tc, int h, int w) {
   int c0 = c_lo;
   for (; c0 + 32 <= c_hi; c0 += 32) {
     float v[32];
     result_chunk<32>(p, s, taddr, c0, n0, valid, vox, v);
-    if (valid) emit_chunk<32>(p, s, c0, n0, tc, h, w, vox, rs, v);
+    if (valid) emit_chunk<32>(p, c0, n0, tc, h, w, vox, v);
   }
   if (c0 < c_hi) {
     float v[16];
     result_chunk<16>(p, s, taddr, c0, n0, valid, vox, v);
-    if (valid) emit_chunk<16>(p, s, c0, n0, tc, h, w, vox, rs, v);
+    if (valid) emit_chunk<16>(p, c0, n0, tc, h, w, vox, v);
   }
 }
 
@@ -419,7 +495,6 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
   const int q = warp & 3;           // TMEM lane quarter this warp may access
   const int grp = (warp - 2) >> 2;  // epilogue group 0 or 1
   const int row = q * 32 + lane;
-  const int hl = row / kTileW, wl = row % kTileW;
   const float rootC = sqrtf(static_cast<float>(p.cout));
   const bool split_cols = p.S == 1;
   const int half = p.BN / 2;
@@ -440,7 +515,9 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
     const TileCoord tc = decode_tile(p, tile, crank);
     const int n0 = tc.n_tile * p.BN;
     for (int sub = split_cols ? 0 : grp; sub < p.S; sub += split_cols ? 1 : 2) {
-      const int h = (tc.th * p.S + sub) * kTileH + hl, w = tc.tw * kTileW + wl;
+      const int idx = sub * kBM + row;  // voxel of the tile, row-major
+      const int h = tc.th * p.tile_rows + idx / p.tile_cols;
+      const int w = tc.tw * p.tile_cols + idx % p.tile_cols;
       const bool valid = h < p.H && w < p.W;
       // output voxel: (t, h, w), or (t, 2h + p', 2w + q') of the 2H x 2W output in phase mode
       const size_t vox = p.phases == 4
@@ -452,9 +529,10 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
                              static_cast<uint32_t>(sub * p.BN);
       const int c_lo = split_cols ? grp * half : 0;
       const int c_hi = split_cols ? c_lo + half : p.BN;
-      float rs = 1.0f;
-      if (p.ep.act != nullptr) {
-        float ss = lane_sumsq(p, s, taddr, c_lo, c_hi, n0, valid, vox);
+      if (p.ep.act == nullptr) {
+        lane_emit(p, s, taddr, c_lo, c_hi, n0, valid, vox, tc, h, w);
+      } else {
+        float ss = lane_pass1(p, s, taddr, c_lo, c_hi, n0, valid, vox);
         if (p.nsplit == 2) {
           // the other half of the channels is in the peer CTA: swap partial sums
           const int slot = (ti & 1u) * 256 + sub * 128 + row;
@@ -487,9 +565,9 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
           __syncwarp();
           ss += part[(grp ^ 1) * 128 + row];
         }
-        rs = rootC / fmaxf(sqrtf(ss), p.ep.eps);
+        const float rs = rootC / fmaxf(sqrtf(ss), p.ep.eps);
+        lane_pass2(p, s, taddr, c_lo, c_hi, n0, valid, vox, rs);
       }
-      lane_emit(p, s, taddr, c_lo, c_hi, n0, valid, vox, tc, h, w, rs);
     }
     tc_fence_before();
     mbar_arrive(smem_u32(&s.tempty[acc]));
@@ -522,8 +600,9 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
   for (int i = threadIdx.x; i < p.cout_pad; i += blockDim.x) {
     s.bias[i] = p.ep.bias[i] + (p.ep.bias2 != nullptr ? p.ep.bias2[i] : 0.0f);
     if (p.ep.act != nullptr && i < p.cout) {
-      s.gamma[i] = p.ep.gamma[i];
-      s.beta[i] = p.ep.beta[i];
+      // halved for silu_half
+      s.gamma[i] = 0.5f * p.ep.gamma[i];
+      s.beta[i] = 0.5f * p.ep.beta[i];
     }
   }
   if (warp == 1) {
@@ -546,14 +625,16 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
     if (lane == 0) producer(p, s, crank);
   } else if (warp == 1) {
     if (lane == 0) {
-      if (p.BN > 256)
-        mma_issuer<1, 2>(p, s, tmem_base);
+      if (p.rowhalo)
+        mma_issuer<2, 1, 3>(p, s, tmem_base);
+      else if (p.BN > 256)
+        mma_issuer<1, 2, 1>(p, s, tmem_base);
       else if (p.S == 1)
-        mma_issuer<1, 1>(p, s, tmem_base);
+        mma_issuer<1, 1, 1>(p, s, tmem_base);
       else if (p.S == 2)
-        mma_issuer<2, 1>(p, s, tmem_base);
+        mma_issuer<2, 1, 1>(p, s, tmem_base);
       else
-        mma_issuer<4, 1>(p, s, tmem_base);
+        mma_issuer<4, 1, 1>(p, s, tmem_base);
     }
   } else {
     epilogue(p, s, tmem_base, warp, lane, crank);
@@ -572,15 +653,15 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
 
 }  // namespace
 
-size_t conv_tc_smem_bytes(int BN, int S, int stages) {
-  const size_t stage = static_cast<size_t>(kBM) * S * kBK * 2 + static_cast<size_t>(BN) * kBK * 2;
+size_t conv_tc_smem_bytes(const ConvParams& p, int stages) {
+  const size_t stage = static_cast<size_t>(conv_tc_a_bytes(p)) + conv_tc_b_bytes(p);
   return 1024 + stages * stage + kCtrlBytes;
 }
 
-int conv_tc_stages_for(int BN, int S) {
+int conv_tc_stages_for(const ConvParams& p) {
   const size_t limit = 232448;  // 227 KB opt-in dynamic shared memory per block
   int st = kMaxStages;
-  while (st > 2 && conv_tc_smem_bytes(BN, S, st) > limit) --st;
+  while (st > 2 && conv_tc_smem_bytes(p, st) > limit) --st;
   return st;
 }
 
@@ -588,7 +669,7 @@ namespace {
 size_t launch_smem(const ConvParams& p) {
   // Every CTA allocates all 512 TMEM columns, so exactly one may live on an SM:
   // ask for more than half of the SM's shared memory even when the ring is small.
-  size_t smem = conv_tc_smem_bytes(p.BN, p.S, p.stages);
+  size_t smem = conv_tc_smem_bytes(p, p.stages);
   if (smem < 120 * 1024) smem = 120 * 1024;
   return smem;
 }

@@ -11,9 +11,10 @@ namespace wvae {
 
 // ----------------------------------------------------------- conv (tcgen05)
 // MMA sub-tile: 128 voxels of one frame, 8 rows x 16 columns (MMA row m =
-// 16 * row + column).  A CTA tile stacks S sub-tiles (8S rows x 16 columns),
-// whose S M=128 MMAs share each weight tile.  K block: 64 input channels of
-// one tap.
+// 16 * row + column).  A CTA tile of tile_rows x tile_cols voxels (128 S in
+// all, tile_cols in {16, 32, 64}) is S such sub-tiles of 128 consecutive
+// voxels in row-major order; their S M=128 MMAs share each weight tile.  K
+// block: 64 input channels of one tap.
 constexpr int kTileH = 8;
 constexpr int kTileW = 16;
 constexpr int kBM = kTileH * kTileW;  // 128
@@ -37,7 +38,7 @@ struct ConvEpilogue {
 };
 
 struct ConvParams {
-  CUtensorMap tmA;   // main input, bf16 [T][H][W][cin_pad], box {64, 16, 8S, 1}
+  CUtensorMap tmA;   // main input, bf16 [T][H][W][cin_pad], box {64, tile_cols, tile_rows, 1}
   CUtensorMap tmB;   // main weights, bf16 [cout_pad][taps * cin_pad], box {64, <=256}
   CUtensorMap tmC;   // cached frames, bf16 [KT-1][H][W][cin_pad], box as tmA (has_cache)
   CUtensorMap tmA2;  // shortcut input, bf16 [T][H][W][cin2_pad], box as tmA (cin2_pad > 0)
@@ -52,15 +53,29 @@ struct ConvParams {
   int has_cache;
   int BN, n_tiles;
   int S;             // MMA sub-tiles per CTA tile; S * BN <= 512 TMEM columns
-  int tiles_w, tiles_h, m_tiles, num_tiles;  // CTA tiles of 8S rows x 16 columns
+  int tile_rows, tile_cols;  // CTA tile, tile_rows * tile_cols = 128 S voxels of one frame
+  int tile_cols_log2;
+  int rowhalo;       // 1: a K block is (kt, kw, 64 channels) with all KH row taps inside:
+                     //    one A box of tile_rows + KH - 1 rows, KH weight tiles; the row
+                     //    tap selects a row offset of the A operand (small BN only)
+  int tiles_w, tiles_h, m_tiles, num_tiles;
   int stages, num_acc;
   int kblocks_main, kblocks;
   ConvEpilogue ep;
   unsigned* err;
 };
 
-size_t conv_tc_smem_bytes(int BN, int S, int stages);
-int conv_tc_stages_for(int BN, int S);
+// Shared-memory bytes of one ring stage's A part (1024-aligned) and B part.
+__host__ __device__ inline uint32_t conv_tc_a_bytes(const ConvParams& p) {
+  const uint32_t rows = p.rowhalo ? static_cast<uint32_t>(p.tile_rows + p.KH - 1)
+                                  : static_cast<uint32_t>(p.tile_rows);
+  return (rows * static_cast<uint32_t>(p.tile_cols) * 128u + 1023u) & ~1023u;
+}
+__host__ __device__ inline uint32_t conv_tc_b_bytes(const ConvParams& p) {
+  return static_cast<uint32_t>(p.rowhalo ? p.KH : 1) * static_cast<uint32_t>(p.BN) * 128u;
+}
+size_t conv_tc_smem_bytes(const ConvParams& p, int stages);
+int conv_tc_stages_for(const ConvParams& p);
 // Clusters of 2 that fit on the device at once (nsplit = 2 launches), 0 on error.
 int conv_tc_max_clusters(const ConvParams& p);
 cudaError_t launch_conv_tc(const ConvParams& p, int grid, cudaStream_t stream);

@@ -8,14 +8,22 @@
 // into one pass; FastVideo Wan2.2 VAE decoder README, "Limits": fp32 norm
 // statistics.)
 //
-// HBM-bound: one read and one write of the tensor.  A group of L lanes owns a
-// voxel (L = 32 for C >= 256); each lane moves 16-byte vectors (8 bf16 / 4 fp32
-// channels), so a warp's accesses to a voxel are one contiguous, fully
-// coalesced run.  Each warp first issues the loads of U voxel groups (kept
-// packed in registers), then reduces the sums of squares with shuffles inside
-// each group and writes the results.  A lane's channels never change, so its
-// gamma/beta live in registers for the whole kernel.  The grid is persistent:
-// exactly the blocks that fit on the GPU at once.
+// HBM-bound: one read and one write of the tensor, and the bf16 path also
+// close to the SM's issue and SFU limits (about 12 elements per SM clock at
+// full HBM rate), so SiLU costs one SFU operation (tanh form) per element.
+//
+// bf16 (norm_silu_ring_kernel): one persistent CTA per SM.  Warp 0 streams
+// contiguous chunks of whole voxels (about 32 KB: the activation is
+// channels-last, so a chunk is one byte range) into a ring of shared-memory
+// stages with bulk asynchronous copies, keeping ~190 KB per SM in flight
+// without holding registers; 16 consumer warps take the voxels of each chunk.
+// A group of L lanes owns a voxel (L = 32 for C >= 256) and moves 16-byte
+// vectors, so shared-memory reads and global writes of a voxel are contiguous
+// runs.  A lane's channels never change: its gamma/beta (pre-halved for the
+// tanh form of SiLU) live in registers for the whole kernel.
+//
+// fp32 (norm_silu_kernel, the reference path): each warp issues the loads of
+// U voxel groups into registers, reduces, and writes; exact SiLU.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -108,7 +116,7 @@ __global__ void __launch_bounds__(kNormThreads, (VEC == 8 && CH <= 4) ? 3 : 2) n
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
           const float s = v[e] * r * g[k][e] + b[k][e];
-          o[e] = (VEC == 8) ? silu_fast(s) : silu_exact(s);
+          o[e] = silu_exact(s);
         }
         uint4 w;
         if constexpr (VEC == 8) {
@@ -122,6 +130,142 @@ __global__ void __launch_bounds__(kNormThreads, (VEC == 8 && CH <= 4) ? 3 : 2) n
       }
     }
   }
+}
+
+// ------------------------------------------------------- bf16: TMA-fed ring
+constexpr int kRingWarps = 16;                       // consumer warps
+constexpr int kRingThreads = 32 * (1 + kRingWarps);  // + the copy warp
+constexpr int kRingStages = 6;
+constexpr int kRingChunkBytes = 32768;
+
+template <int CH>
+__global__ void __launch_bounds__(kRingThreads, 1)
+    norm_silu_ring_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* y,
+                          const float* __restrict__ gamma, const float* __restrict__ beta,
+                          long nvox, int C, int L, int vpc, float eps, unsigned* err) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  const uint32_t chunk_bytes = static_cast<uint32_t>(vpc) * C * 2;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + kRingStages * chunk_bytes);
+  uint64_t* empty = full + kRingStages;
+  int* abort_flag = reinterpret_cast<int*>(empty + kRingStages);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kRingStages; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), kRingWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const long nchunks = (nvox + vpc - 1) / vpc;
+
+  if (warp == 0) {
+    if (lane != 0) return;
+    uint32_t it = 0;
+    for (long ch = blockIdx.x; ch < nchunks; ch += gridDim.x, ++it) {
+      const uint32_t st = it % kRingStages, ph = (it / kRingStages) & 1u;
+      if (!mbar_wait_bounded(smem_u32(&empty[st]), ph ^ 1u, abort_flag, err,
+                             DEVERR_TIMEOUT_PRODUCER))
+        break;
+      const long v0 = ch * vpc;
+      const long nv = nvox - v0 < vpc ? nvox - v0 : vpc;
+      const uint32_t bytes = static_cast<uint32_t>(nv) * C * 2;
+      mbar_arrive_expect_tx(smem_u32(&full[st]), bytes);
+      bulk_load(smem_u32(smem_raw + st * chunk_bytes), x + v0 * C, bytes, smem_u32(&full[st]));
+    }
+    // Do not leave while copies issued by this thread may still be landing.
+    for (uint32_t st = 0; st < static_cast<uint32_t>(kRingStages) && st < it; ++st) {
+      const uint32_t last = st + ((it - 1 - st) / kRingStages) * kRingStages;
+      volatile int never = 0;
+      mbar_wait_bounded(smem_u32(&full[st]), (last / kRingStages) & 1u, &never, err,
+                        DEVERR_TIMEOUT_DRAIN, kDrainLimitNs);
+    }
+    return;
+  }
+
+  const int cw = warp - 1;
+  const int sub = lane % L, grp = lane / L, gpw = 32 / L;
+  const int nvec = C / 8;
+  float g[CH][8], b[CH][8];
+#pragma unroll
+  for (int k = 0; k < CH; ++k) {
+    const int vi = sub + k * L;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      g[k][e] = vi < nvec ? 0.5f * __ldg(gamma + vi * 8 + e) : 0.0f;
+      b[k][e] = vi < nvec ? 0.5f * __ldg(beta + vi * 8 + e) : 0.0f;
+    }
+  }
+  const float rootC = sqrtf(static_cast<float>(C));
+  uint32_t it = 0;
+  for (long ch = blockIdx.x; ch < nchunks; ch += gridDim.x, ++it) {
+    const uint32_t st = it % kRingStages, ph = (it / kRingStages) & 1u;
+    int ok = 0;
+    if (lane == 0)
+      ok = mbar_wait_bounded(smem_u32(&full[st]), ph, abort_flag, err, DEVERR_TIMEOUT_EPILOGUE)
+               ? 1
+               : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) break;
+    __syncwarp();
+    const long v0 = ch * vpc;
+    const int nv = nvox - v0 < vpc ? static_cast<int>(nvox - v0) : vpc;
+    const uint8_t* stage = smem_raw + st * chunk_bytes;
+    // warp-uniform bound: the shuffles need every lane
+    for (int vb = cw * gpw; vb < nv; vb += kRingWarps * gpw) {
+      const int vl = vb + grp;
+      const bool live = vl < nv;
+      const uint4* src = reinterpret_cast<const uint4*>(stage + static_cast<size_t>(vl) * C * 2);
+      uint4 raw[CH];
+      float ss = 0.0f;
+#pragma unroll
+      for (int k = 0; k < CH; ++k) {
+        const int vi = sub + k * L;
+        raw[k] = (live && vi < nvec) ? src[vi] : make_uint4(0u, 0u, 0u, 0u);
+        float v[8];
+        unpack<8>(raw[k], v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
+      }
+      for (int off = L >> 1; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      const float r = rootC / fmaxf(sqrtf(ss), eps);
+      uint4* dst = reinterpret_cast<uint4*>(y + (v0 + vl) * C);
+#pragma unroll
+      for (int k = 0; k < CH; ++k) {
+        const int vi = sub + k * L;
+        if (!live || vi >= nvec) continue;
+        float v[8], o[8];
+        unpack<8>(raw[k], v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = silu_half(fmaf(v[e], r * g[k][e], b[k][e]));
+        uint4 w;
+        w.x = pack_bf16x2(o[0], o[1]); w.y = pack_bf16x2(o[2], o[3]);
+        w.z = pack_bf16x2(o[4], o[5]); w.w = pack_bf16x2(o[6], o[7]);
+        dst[vi] = w;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&empty[st]));
+  }
+}
+
+template <int CH>
+cudaError_t launch_ring(const __nv_bfloat16* x, __nv_bfloat16* y, const float* gamma,
+                        const float* beta, long nvox, int C, int L, float eps, int num_sms,
+                        cudaStream_t stream) {
+  int vpc = kRingChunkBytes / (C * 2);
+  if (vpc < 1) vpc = 1;
+  const size_t smem = static_cast<size_t>(kRingStages) * vpc * C * 2 + 2 * kRingStages * 8 + 16;
+  auto kern = norm_silu_ring_kernel<CH>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const long nchunks = (nvox + vpc - 1) / vpc;
+  const int grid = nchunks < num_sms ? static_cast<int>(nchunks) : num_sms;
+  kern<<<grid, kRingThreads, smem, stream>>>(x, y, gamma, beta, nvox, C, L, vpc, eps,
+                                             device_error_word());
+  return cudaGetLastError();
 }
 
 template <typename T, int VEC, int CH, int U>
@@ -162,7 +306,14 @@ cudaError_t launch_impl(const T* x, T* y, const float* gamma, const float* beta,
 cudaError_t launch_norm_silu_bf16(const __nv_bfloat16* x, __nv_bfloat16* y, const float* gamma,
                                   const float* beta, long nvox, int C, float eps, int num_sms,
                                   cudaStream_t stream) {
-  return launch_impl<__nv_bfloat16, 8>(x, y, gamma, beta, nvox, C, eps, num_sms, stream);
+  const int nvec = C / 8;
+  int L = 1;
+  while (L < nvec && L < 32) L <<= 1;
+  const int ch = (nvec + L - 1) / L;
+  if (ch == 1) return launch_ring<1>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
+  if (ch == 2) return launch_ring<2>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
+  if (ch <= 4) return launch_ring<4>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_norm_silu_f32(const float* x, float* y, const float* gamma, const float* beta,
