@@ -39,9 +39,10 @@ def test_conv_kernel_sizes_two_chunks(k):
     assert_close(from_cl(y), O.causal_conv3d(x, w, b), torch.bfloat16, f"k={k}")
 
 
-@pytest.mark.parametrize("dtype,cout", [(torch.bfloat16, 64), (torch.float32, 64), (torch.bfloat16, 128)])
+@pytest.mark.parametrize("dtype,cout", [(torch.bfloat16, 64), (torch.float32, 64), (torch.bfloat16, 128), (torch.bfloat16, 16)])
 def test_conv_with_residual_norm_and_cache(dtype, cout):
-    """cout = 64 runs the row-halo main loop (one A load per (kt, kw) window)."""
+    """cout 64 and 128: a group's window and its three row taps in one stage;
+    cout 16: the column taps ride in N (the residual case runs the plain path)."""
     bf = dtype == torch.bfloat16
     x, w, b = synth.conv_input(cin=64, cout=cout, T=3, H=10, W=18, seed=11, bf16=bf)
     g = torch.Generator().manual_seed(12)

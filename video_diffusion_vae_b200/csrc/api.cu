@@ -188,12 +188,20 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   }
   p.n_tiles = L.cout_pad / p.BN;
   // Sub-tiles per CTA tile: S M=128 MMAs share each weight tile (see conv_tc.cu).
-  p.S = p.BN >= 512 ? 1 : (p.BN >= 128 ? 2 : 4);
-  // Narrow layers (the head) are bound by refilling A once per tap: load each
-  // (kt, kw) window once with its row halo and run the KH row taps from it.
-  p.rowhalo = (p.BN <= 64 && a.KH == 3 && a.phases == 1 && a.cin2_pad == 0 && p.nsplit == 1) ? 1 : 0;
-  if (p.rowhalo) p.S = 2;
-  p.num_acc = 2 * p.S * p.BN <= 512 ? 2 : 1;
+  p.S = 2;
+  // At 16 output channels (the head) a tcgen05.mma is mostly fixed issue
+  // cost, so the three column taps ride in N (N = 48) and the epilogue adds
+  // each tap's partial sum from the neighbouring column's TMEM lane.
+  const bool kwn = p.BN == 16 && a.KH == 3 && a.KW == 3 && a.phases == 1 && a.cin2_pad == 0 &&
+                   a.ep.act == nullptr && a.ep.residual == nullptr && p.nsplit == 1;
+  p.nw = kwn ? a.KW : 1;
+  p.num_acc = 2 * p.S * static_cast<int>(conv_tc_acc_stride(p)) <= 512 ? 2 : 1;
+  // Row taps share one A window (the tile plus its row halo) per (kt, kw); up
+  // to 128 output channels a B stage carries all of a window's row taps.
+  p.kh_eff = a.phases == 4 ? 2 : a.KH;
+  p.kw_eff = a.phases == 4 ? 2 : (kwn ? 1 : a.KW);
+  p.b_tiles = (p.BN <= 128 || p.kh_eff == 1) ? p.kh_eff : 1;
+  p.combined = p.b_tiles == p.kh_eff ? 1 : 0;
   // Tile shape: 128 S voxels as tile_rows x tile_cols, tile_cols in {16, 32,
   // 64}; the narrowest shape among those needing the fewest waves of tiles over
   // the CTAs (or CTA pairs) that run at once.
@@ -205,20 +213,24 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   };
   p.tile_cols = kTileW;
   p.tile_rows = kBM * p.S / kTileW;
-  for (int cols = 2 * kTileW; cols <= 64 && kBM * p.S / cols >= kTileH; cols *= 2) {
-    if (waves(kBM * p.S / cols, cols) < waves(p.tile_rows, p.tile_cols)) {
-      p.tile_cols = cols;
-      p.tile_rows = kBM * p.S / cols;
+  if (!kwn) {
+    for (int cols = 2 * kTileW; cols <= 64 && kBM * p.S / cols >= kTileH; cols *= 2) {
+      if (waves(kBM * p.S / cols, cols) < waves(p.tile_rows, p.tile_cols)) {
+        p.tile_cols = cols;
+        p.tile_rows = kBM * p.S / cols;
+      }
     }
   }
-  p.tile_cols_log2 = p.tile_cols == 16 ? 4 : (p.tile_cols == 32 ? 5 : 6);
-  p.stages = conv_tc_stages_for(p);
-  p.tiles_w = (a.W + p.tile_cols - 1) / p.tile_cols;
+  // with the column taps in N the two edge columns of a tile only feed their
+  // neighbours: 16 computed columns give 14 outputs
+  p.out_cols = kwn ? p.tile_cols - 2 : p.tile_cols;
+  conv_tc_choose_stages(p);
+  p.tiles_w = (a.W + p.out_cols - 1) / p.out_cols;
   p.tiles_h = (a.H + p.tile_rows - 1) / p.tile_rows;
   p.m_tiles = a.T * p.tiles_h * p.tiles_w;
   p.num_tiles = p.m_tiles * per_m;
-  p.kblocks_main = (p.rowhalo ? a.KT * a.KW : a.KT * a.KH * a.KW) * (a.cin_pad / kBK);
-  p.kblocks = p.kblocks_main + a.cin2_pad / kBK;
+  p.groups_main = (a.phases == 4 ? 1 : a.KT) * p.kw_eff * (a.cin_pad / kBK);
+  p.groups = p.groups_main + a.cin2_pad / kBK;
   a.ep.bias = reinterpret_cast<const float*>(static_cast<const char*>(a.packed) + L.bias_off);
   if (a.packed2 != nullptr) {
     const PackedLayout L2 = packed_layout(a.cout, a.cin2_pad, 1, 1, 1, WVAE_BF16);
@@ -226,8 +238,8 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   }
   p.ep = a.ep;
   p.err = d.err;
-  const int box_rows = p.BN > 256 ? 256 : p.BN;
-  const int a_rows = p.rowhalo ? p.tile_rows + a.KH - 1 : p.tile_rows;
+  const int box_rows = p.BN;  // BN <= 256
+  const int a_rows = static_cast<int>(conv_tc_a_rows(p));
   if (!encode_act(&p.tmA, a.x, a.cin_pad, a.W, a.H, a.T, p.tile_cols, a_rows))
     return WVAE_ERR_CUDA;
   if (!encode_weights(&p.tmB, a.packed, L.taps * a.cin_pad, L.cout_pad, box_rows))

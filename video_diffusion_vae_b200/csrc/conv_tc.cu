@@ -6,9 +6,9 @@
 //   A[m, (tap, i)] = a[t + kt - (KT-1), h + kh - (KH-1)/2, w + kw - (KW-1)/2, i]
 //
 // The causal front frames and the spatial border are zero (or, for t' < 0, the
-// previous chunk's cached frames).  No padded copy exists: every K block is one
-// TMA box load of the channels-last activation at the tap-shifted coordinates,
-// and the tensor map's out-of-bounds fill supplies the zeros.  (Conv definition:
+// previous chunk's cached frames).  No padded copy exists: every A load is one
+// TMA box of the channels-last activation at tap-shifted coordinates, and the
+// tensor map's out-of-bounds fill supplies the zeros.  (Conv definition:
 // FastVideo "Wan2.2 VAE decoder (sm_100a, sm_103a)" README, "Limits": bf16
 // operands, fp32 accumulation; temporal caching: TensorRT-LLM issue #19309,
 // "Feature, motivation and proposed scope".)
@@ -16,18 +16,24 @@
 // One CTA per SM, persistent over output tiles of tile_rows x tile_cols voxels
 // of one frame (128 S voxels: S MMA sub-tiles of 128 consecutive voxels in
 // row-major order; the shape is chosen per layer to balance the waves) x BN
-// output channels.  Warp roles:
-//   warp 0      TMA producer: A box {64 ch, tile_cols w, tile_rows h, 1 t} +
-//               B box {64, BN} per K block into a ring of `stages` stages;
-//   warp 1      MMA issuer: per K block, 4 K steps x S sub-tiles of
-//               tcgen05.mma (M=128, N=BN<=256, K=16) sharing the weight tile,
-//               into TMEM (two accumulators when 2 S BN <= 512, so the
-//               epilogue of tile i overlaps the main loop of tile i+1);
+// output channels.  The reduction runs in K groups (kt, column tap kw, 64
+// input channels).  Warp roles:
+//   warp 0      TMA producer: per group one A window {64 ch, tile_cols w,
+//               tile_rows + KH - 1 h, 1 t} (the tile plus its row-tap halo)
+//               into the A ring, and the KH weight tiles {64, BN} of the
+//               group's row taps into the B ring;
+//   warp 1      MMA issuer: per weight tile (row tap kh), 4 K steps x S
+//               sub-tiles of tcgen05.mma (M=128, N=BN<=256, K=16) whose A
+//               operand starts kh tile rows into the window (whole 8-row
+//               swizzle atoms, so no copy), into TMEM (two accumulators when
+//               2 S BN <= 512: the epilogue of tile i overlaps the main loop
+//               of tile i+1);
 //   warps 2..9  epilogue, two groups of 4 warps (one warp per TMEM lane
-//               quarter each): one TMEM lane = one output voxel per thread;
-//               with S >= 2 the groups take alternate sub-tiles, with S = 1
-//               each takes half of the channels (the two halves of the RMS
-//               sum meet in shared memory).
+//               quarter each) taking alternate sub-tiles: one TMEM lane = one
+//               output voxel per thread.
+// The conv is bound by how fast L2 can refill shared memory, so the operand
+// bytes per MMA FLOP decide the speed: the row-tap windows load each input
+// row about once per (kt, kw) instead of once per tap.
 // 512 output channels with the next layer's norm fused: a cluster of two CTAs
 // splits N (each runs the S = 2, BN = 256 main loop on its half of the
 // channels for the same M tiles) and the two epilogues exchange each voxel's
@@ -49,18 +55,17 @@ namespace wvae {
 namespace {
 
 struct Smem {
-  uint8_t* stages;        // stage s at stages + s * stage_bytes, 1024-aligned
-  uint32_t stage_bytes;
-  uint32_t a_bytes;
-  uint32_t tx_bytes;      // bytes the TMA loads of one main-loop stage deliver
-  uint64_t* full;         // [kMaxStages]
-  uint64_t* empty;        // [kMaxStages]
+  uint8_t* a_ring;        // A stage i at a_ring + i * a_bytes, 1024-aligned
+  uint8_t* b_ring;        // B stage j at b_ring + j * b_bytes, 1024-aligned
+  uint32_t a_bytes, b_bytes;
+  uint64_t* full_a;       // [kMaxStages]
+  uint64_t* empty_a;      // [kMaxStages]
+  uint64_t* full_b;       // [kMaxStages]
+  uint64_t* empty_b;      // [kMaxStages]
   uint64_t* tfull;        // [2]
   uint64_t* tempty;       // [2]
   uint64_t* drain;        // [1]
-  uint64_t* ssbar;        // [1] the two epilogue groups' partial RMS sums are written
   uint64_t* xbar;         // [2] (per tile parity) the peer CTA's partial sums have arrived
-  float* ss_part;         // [2 tile parities][2 groups][128 rows]
   float* xpart;           // [2 tile parities][256]: partial sums written by the peer CTA
   uint32_t* tmem_slot;
   int* abort_flag;
@@ -69,7 +74,7 @@ struct Smem {
   float* beta;            // [512]
 };
 
-constexpr uint32_t kCtrlBytes = 512 + 3 * 512 * 4 + 2 * 2 * 128 * 4 + 2 * 256 * 4;
+constexpr uint32_t kCtrlBytes = 512 + 3 * 512 * 4 + 2 * 256 * 4;
 
 __device__ __forceinline__ Smem carve(uint8_t* raw, const ConvParams& p) {
   Smem s;
@@ -77,26 +82,24 @@ __device__ __forceinline__ Smem carve(uint8_t* raw, const ConvParams& p) {
   uint32_t pad = (1024u - (base & 1023u)) & 1023u;
   uint8_t* al = raw + pad;
   s.a_bytes = conv_tc_a_bytes(p);
-  s.stage_bytes = s.a_bytes + conv_tc_b_bytes(p);
-  s.tx_bytes = (p.rowhalo ? static_cast<uint32_t>(p.tile_rows + p.KH - 1) : static_cast<uint32_t>(p.tile_rows)) *
-                   static_cast<uint32_t>(p.tile_cols) * 128u +
-               conv_tc_b_bytes(p);
-  s.stages = al;
-  uint8_t* ctrl = al + p.stages * s.stage_bytes;
-  s.full = reinterpret_cast<uint64_t*>(ctrl);
-  s.empty = s.full + kMaxStages;
-  s.tfull = s.empty + kMaxStages;
+  s.b_bytes = conv_tc_b_bytes(p);
+  s.a_ring = al;
+  s.b_ring = al + p.stages_a * s.a_bytes;
+  uint8_t* ctrl = s.b_ring + p.stages_b * s.b_bytes;
+  s.full_a = reinterpret_cast<uint64_t*>(ctrl);
+  s.empty_a = s.full_a + kMaxStages;
+  s.full_b = s.empty_a + kMaxStages;
+  s.empty_b = s.full_b + kMaxStages;
+  s.tfull = s.empty_b + kMaxStages;
   s.tempty = s.tfull + 2;
   s.drain = s.tempty + 2;
-  s.ssbar = s.drain + 1;
-  s.xbar = s.ssbar + 1;
+  s.xbar = s.drain + 1;
   s.tmem_slot = reinterpret_cast<uint32_t*>(s.xbar + 2);
   s.abort_flag = reinterpret_cast<int*>(s.tmem_slot + 1);
   s.bias = reinterpret_cast<float*>(ctrl + 512);
   s.gamma = s.bias + 512;
   s.beta = s.gamma + 512;
-  s.ss_part = s.beta + 512;
-  s.xpart = s.ss_part + 2 * 2 * 128;
+  s.xpart = s.beta + 512;
   return s;
 }
 
@@ -135,82 +138,110 @@ __device__ __forceinline__ int tile_stride(const ConvParams& p) {
   return p.nsplit == 2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 }
 
+// Waits, bounded, until every copy this thread issued into a ring has landed.
+__device__ void drain_ring(const uint64_t* full, uint32_t issued, int stages, unsigned* err) {
+  for (uint32_t st = 0; st < static_cast<uint32_t>(stages) && st < issued; ++st) {
+    const uint32_t last = st + ((issued - 1 - st) / stages) * stages;
+    volatile int never = 0;
+    mbar_wait_bounded(smem_u32(&full[st]), (last / stages) & 1u, &never, err, DEVERR_TIMEOUT_DRAIN,
+                      kDrainLimitNs);
+  }
+}
+
+// K group = (kt, column tap kw, 64 input channels): one A window holding the
+// tile's rows plus the row-tap halo goes to the A ring, then the kh_eff weight
+// tiles of taps (kt, 0..kh_eff-1, kw) to the B ring, b_tiles per stage.  A
+// second-segment group (1x1x1 shortcut) is one A tile without halo and one
+// weight tile (alone in its B stage).
 __device__ void producer(const ConvParams& p, const Smem& s, int crank) {
   const int cchunks = p.cin_pad / kBK;
-  const int kwkh = p.KH * p.KW;
-  const int b_rows = p.BN > 256 ? 256 : p.BN;
-  const int b_loads = p.BN > 256 ? 2 : 1;
-  const uint32_t b_box_bytes = static_cast<uint32_t>(b_rows) * kBK * 2;
-  uint32_t it = 0;
+  const uint32_t a_tx_main = conv_tc_a_rows(p) * static_cast<uint32_t>(p.tile_cols) * 128u;
+  const uint32_t a_tx_sc = static_cast<uint32_t>(p.tile_rows * p.tile_cols) * 128u;
+  const uint32_t tile_tx = static_cast<uint32_t>(p.BN) * 128u;
+  const int kw_stride = p.kw_eff * p.nw;  // tap = ((kt kh_eff + kh) kw_stride + kw) (+ phase)
+  uint32_t ia = 0, ib = 0;
   bool aborted = false;
   for (int tile = tile_first(p); tile < p.num_tiles && !aborted; tile += tile_stride(p)) {
     const TileCoord tc = decode_tile(p, tile, crank);
-    const int h0 = tc.th * p.tile_rows, w0 = tc.tw * p.tile_cols;
-    for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
-      const uint32_t st = it % p.stages;
-      const uint32_t ph = (it / p.stages) & 1u;
-      if (!mbar_wait_bounded(smem_u32(&s.empty[st]), ph ^ 1u, s.abort_flag, p.err,
-                             DEVERR_TIMEOUT_PRODUCER)) {
-        aborted = true;
-        break;
-      }
-      const uint32_t bar = smem_u32(&s.full[st]);
-      const uint32_t a_dst = smem_u32(s.stages + st * s.stage_bytes);
-      const uint32_t b_dst = a_dst + s.a_bytes;
-      if (p.rowhalo && kb < p.kblocks_main) {
-        // (kt, kw, channel chunk): rows h0 - (KH-1)/2 .. h0 + tile_rows + KH/2 once,
-        // the KH row taps' weight tiles side by side
-        mbar_arrive_expect_tx(bar, s.tx_bytes);
-        const int tap2 = kb / cchunks, cc = kb - tap2 * cchunks;
-        const int kt = tap2 / p.KW, kw = tap2 - kt * p.KW;
-        const int ts = tc.t + kt - (p.KT - 1);
-        const int hs = h0 - (p.KH - 1) / 2, ws = w0 + kw - (p.KW - 1) / 2;
-        if (ts < 0 && p.has_cache)
-          tma_load_4d(a_dst, &p.tmC, bar, cc * kBK, ws, hs, ts + p.KT - 1);
-        else
-          tma_load_4d(a_dst, &p.tmA, bar, cc * kBK, ws, hs, ts);
-        for (int kh = 0; kh < p.KH; ++kh) {
-          const int tap = (kt * p.KH + kh) * p.KW + kw;
-          tma_load_2d(b_dst + kh * static_cast<uint32_t>(p.BN) * 128u, &p.tmB, bar,
-                      tap * p.cin_pad + cc * kBK, tc.n_tile * p.BN);
-        }
-        continue;
-      }
-      mbar_arrive_expect_tx(bar, s.tx_bytes);
-      if (kb < p.kblocks_main) {
-        const int tap = kb / cchunks, cc = kb - tap * cchunks;
-        const int kt = tap / kwkh, r = tap - kt * kwkh;
-        const int kh = r / p.KW, kw = r - kh * p.KW;
-        const int ts = tc.t + kt - (p.KT - 1);
-        // phase mode: output (2h+p', 2w+q') reads input rows h + kh + p' - 1
-        const int oh = p.phases == 4 ? (tc.phase >> 1) - 1 : -(p.KH - 1) / 2;
-        const int ow = p.phases == 4 ? (tc.phase & 1) - 1 : -(p.KW - 1) / 2;
-        const int hs = h0 + kh + oh;
-        const int ws = w0 + kw + ow;
-        if (ts < 0 && p.has_cache)
-          tma_load_4d(a_dst, &p.tmC, bar, cc * kBK, ws, hs, ts + p.KT - 1);
-        else
-          tma_load_4d(a_dst, &p.tmA, bar, cc * kBK, ws, hs, ts);
-        const int kcoord = (tc.phase * 4 * (p.phases == 4) + tap) * p.cin_pad + cc * kBK;
-        for (int l = 0; l < b_loads; ++l)
-          tma_load_2d(b_dst + l * b_box_bytes, &p.tmB, bar, kcoord, tc.n_tile * p.BN + l * 256);
+    const int h0 = tc.th * p.tile_rows, w0 = tc.tw * p.out_cols;
+    // output (h, w) reads input row h + oh + kh and column w + ow + kw; phase
+    // mode: output (2h+p', 2w+q') reads rows h + p' - 1 + r, columns w + q' - 1 + c
+    const int oh = p.phases == 4 ? (tc.phase >> 1) - 1 : -(p.KH - 1) / 2;
+    const int ow = p.phases == 4 ? (tc.phase & 1) - 1 : -(p.KW - 1) / 2;
+    const int tap0 = p.phases == 4 ? tc.phase * 4 : 0;
+    for (int g = 0; g < p.groups; ++g) {
+      const bool main_seg = g < p.groups_main;
+      int kt = 0, kw = 0, cc;
+      if (main_seg) {
+        const int tw = g / cchunks;
+        cc = g - tw * cchunks;
+        kt = tw / p.kw_eff;
+        kw = tw - kt * p.kw_eff;
       } else {
-        const int cc = kb - p.kblocks_main;
-        tma_load_4d(a_dst, &p.tmA2, bar, cc * kBK, w0, h0, tc.t);
-        for (int l = 0; l < b_loads; ++l)
-          tma_load_2d(b_dst + l * b_box_bytes, &p.tmB2, bar, cc * kBK, tc.n_tile * p.BN + l * 256);
+        cc = g - p.groups_main;
       }
+      const uint32_t a_tx = main_seg ? a_tx_main : a_tx_sc;
+      // the A window of the group (on its own barrier, or on the B stage's)
+      auto load_a = [&](uint32_t dst, uint32_t bar) {
+        if (main_seg) {
+          const int ts = tc.t + kt - (p.KT - 1);
+          if (ts < 0 && p.has_cache)
+            tma_load_4d(dst, &p.tmC, bar, cc * kBK, w0 + ow + kw, h0 + oh, ts + p.KT - 1);
+          else
+            tma_load_4d(dst, &p.tmA, bar, cc * kBK, w0 + ow + kw, h0 + oh, ts);
+        } else {
+          tma_load_4d(dst, &p.tmA2, bar, cc * kBK, w0, h0, tc.t);
+        }
+      };
+      if (!p.combined) {
+        const uint32_t st = ia % p.stages_a, ph = (ia / p.stages_a) & 1u;
+        if (!mbar_wait_bounded(smem_u32(&s.empty_a[st]), ph ^ 1u, s.abort_flag, p.err,
+                               DEVERR_TIMEOUT_PRODUCER)) {
+          aborted = true;
+          break;
+        }
+        const uint32_t bar = smem_u32(&s.full_a[st]);
+        mbar_arrive_expect_tx(bar, a_tx);
+        load_a(smem_u32(s.a_ring + st * s.a_bytes), bar);
+        ++ia;
+      }
+      const int nkh = main_seg ? p.kh_eff : 1;
+      const int per_stage = main_seg ? p.b_tiles : 1;
+      for (int kh0 = 0; kh0 < nkh; kh0 += per_stage, ++ib) {
+        const uint32_t st = ib % p.stages_b, ph = (ib / p.stages_b) & 1u;
+        if (!mbar_wait_bounded(smem_u32(&s.empty_b[st]), ph ^ 1u, s.abort_flag, p.err,
+                               DEVERR_TIMEOUT_PRODUCER)) {
+          aborted = true;
+          break;
+        }
+        const uint32_t bar = smem_u32(&s.full_b[st]);
+        const uint32_t dst = smem_u32(s.b_ring + st * s.b_bytes);
+        const uint32_t b_tx = main_seg ? s.b_bytes : tile_tx;
+        if (p.combined) {
+          // one stage per group: A slot st travels with B slot st on one barrier
+          mbar_arrive_expect_tx(bar, a_tx + b_tx);
+          load_a(smem_u32(s.a_ring + st * s.a_bytes), bar);
+        } else {
+          mbar_arrive_expect_tx(bar, b_tx);
+        }
+        if (main_seg) {
+          // weight tiles [row tap j][column tap u], BN rows each
+          for (int j = 0; j < per_stage; ++j)
+            for (int u = 0; u < p.nw; ++u) {
+              const int tap = tap0 + (kt * p.kh_eff + kh0 + j) * kw_stride + kw + u;
+              tma_load_2d(dst + (j * p.nw + u) * tile_tx, &p.tmB, bar,
+                          tap * p.cin_pad + cc * kBK, tc.n_tile * p.BN);
+            }
+        } else {
+          tma_load_2d(dst, &p.tmB2, bar, cc * kBK, tc.n_tile * p.BN);
+        }
+      }
+      if (aborted) break;
     }
   }
   // Do not leave while copies issued by this thread may still be landing.
-  const uint32_t issued = it;
-  for (uint32_t st = 0; st < static_cast<uint32_t>(p.stages) && st < issued; ++st) {
-    const uint32_t last = st + ((issued - 1 - st) / p.stages) * p.stages;
-    const uint32_t ph = (last / p.stages) & 1u;
-    volatile int never = 0;
-    mbar_wait_bounded(smem_u32(&s.full[st]), ph, &never, p.err, DEVERR_TIMEOUT_DRAIN,
-                      kDrainLimitNs);
-  }
+  drain_ring(s.full_a, ia, p.stages_a, p.err);
+  drain_ring(s.full_b, ib, p.stages_b, p.err);
 }
 
 // ----------------------------------------------------------------------- MMA
@@ -219,28 +250,36 @@ __device__ __noinline__ bool mma_wait_slow(uint32_t bar, uint32_t parity, volati
   return mbar_wait_bounded(bar, parity, abort_flag, err, DEVERR_TIMEOUT_MMA);
 }
 
-// S sub-tiles and HALVES weight halves are compile-time so the issue loop is
-// fully unrolled: the thread must hand the next MMA to the tensor core as soon
-// as it can take it.  KHT > 1 (row-halo mode): each K step runs the KHT row taps, the A operand
-// shifted down by one tile row (tile_cols voxels, whole 8-row swizzle atoms)
-// and the B operand moved to that tap's weight tile.
-template <int S, int HALVES, int KHT>
+// S sub-tiles, KHT row taps and BT weight tiles per B stage are compile-time
+// so the issue loop is fully unrolled: the thread must hand the next MMA to
+// the tensor core as soon as it can take it.  Per weight tile (row tap kh),
+// 4 K steps x S sub-tiles of M=128 x N=BN x K=16; the A operand of row tap kh
+// starts kh tile rows (kh * tile_cols voxels, whole 8-row swizzle atoms) into
+// the A window.
+__device__ __forceinline__ bool mma_wait(uint32_t bar, uint32_t ph, const Smem& s,
+                                         const ConvParams& p) {
+  return mbar_try_wait(bar, ph) || mma_wait_slow(bar, ph, s.abort_flag, p.err);
+}
+
+// COMBINED: a group's A window and weight tiles share one stage and barrier.
+template <int S, int KHT, int BT, bool COMBINED>
 __device__ void mma_issuer(const ConvParams& p, const Smem& s, uint32_t tmem_base) {
-  const int n_inst = p.BN > 256 ? 256 : p.BN;
-  const uint32_t idesc = umma_idesc_bf16(kBM, n_inst);
-  // Descriptors of stage 0; the start field counts 16-byte units: stage st
-  // adds stage_bytes / 16, sub-tile s adds 16 KB / 16, K step k adds 32 B / 16
-  // and the second weight half 32 KB / 16.
-  const uint64_t adesc0 = umma_desc_sw128(smem_u32(s.stages));
-  const uint64_t bdesc0 = umma_desc_sw128(smem_u32(s.stages) + s.a_bytes);
-  const uint32_t stage_step = s.stage_bytes >> 4;
+  static_assert(BT == 1 || BT == KHT, "a B stage holds one weight tile or the group's row taps");
+  static_assert(!COMBINED || BT == KHT, "a combined stage holds all of a group's weight tiles");
+  const uint32_t n_mma = static_cast<uint32_t>(p.nw * p.BN);  // N of one MMA
+  const uint32_t idesc = umma_idesc_bf16(kBM, static_cast<int>(n_mma));
+  // Descriptors of stage 0 of each ring; the start field counts 16-byte units.
+  const uint64_t adesc0 = umma_desc_sw128(smem_u32(s.a_ring));
+  const uint64_t bdesc0 = umma_desc_sw128(smem_u32(s.b_ring));
+  const uint32_t a_step = s.a_bytes >> 4, b_step = s.b_bytes >> 4;
   const uint32_t sub_step = (static_cast<uint32_t>(kBM) * 128u) >> 4;
-  const uint32_t kh_step_a = static_cast<uint32_t>(p.tile_cols) * 8u;  // tile_cols * 128 B / 16
-  const uint32_t kh_step_b = static_cast<uint32_t>(p.BN) * 8u;
-  const uint32_t full0 = smem_u32(&s.full[0]), empty0 = smem_u32(&s.empty[0]);
-  const uint32_t bn = static_cast<uint32_t>(p.BN);
-  const uint32_t acc_cols = static_cast<uint32_t>(S) * bn;
-  uint32_t st = 0, ph = 0, ai = 0;
+  const uint32_t kh_step = static_cast<uint32_t>(p.tile_cols) * 8u;  // tile_cols * 128 B / 16
+  const uint32_t tap_step = n_mma * 8u;  // one row tap's weight tiles: nw BN * 128 B / 16
+  const uint32_t full_a0 = smem_u32(&s.full_a[0]), empty_a0 = smem_u32(&s.empty_a[0]);
+  const uint32_t full_b0 = smem_u32(&s.full_b[0]), empty_b0 = smem_u32(&s.empty_b[0]);
+  const uint32_t n_stride = conv_tc_acc_stride(p);  // TMEM columns per sub-tile
+  const uint32_t acc_cols = static_cast<uint32_t>(S) * n_stride;
+  uint32_t sa = 0, pa = 0, sb = 0, pb = 0, ai = 0;
   bool aborted = false;
   for (int tile = tile_first(p); tile < p.num_tiles && !aborted; tile += tile_stride(p), ++ai) {
     const uint32_t acc = ai % p.num_acc;
@@ -252,34 +291,63 @@ __device__ void mma_issuer(const ConvParams& p, const Smem& s, uint32_t tmem_bas
     }
     tc_fence_after();
     const uint32_t d_tmem = tmem_base + acc * acc_cols;
-    for (int kb = 0; kb < p.kblocks; ++kb) {
-      const uint32_t bar = full0 + st * 8u;
-      if (!mbar_try_wait(bar, ph) && !mma_wait_slow(bar, ph, s.abort_flag, p.err)) {
+    for (int g = 0; g < p.groups && !aborted; ++g) {
+      if (!COMBINED && !mma_wait(full_a0 + sa * 8u, pa, s, p)) {
         aborted = true;
         break;
       }
-      tc_fence_after();
-      const uint64_t a_st = adesc0 + st * stage_step;
-      const uint64_t b_st = bdesc0 + st * stage_step;
+      const uint64_t a_st = adesc0 + (COMBINED ? sb : sa) * a_step;
+      const uint32_t first = g == 0 ? 0u : 1u;  // the tile's first MMA overwrites
+      // MMAs of row tap kh (A rows kh.., weight tile j of the B stage)
+      auto issue = [&](int kh, int j) {
+        const uint64_t a_kh = a_st + kh * kh_step;
+        const uint64_t b_st = bdesc0 + sb * b_step + j * tap_step;
 #pragma unroll
-      for (int k = 0; k < kBK / 16; ++k) {
+        for (int k = 0; k < kBK / 16; ++k) {
+          const uint32_t accumulate = (k | kh) != 0 ? 1u : first;
+#pragma unroll
+          for (int sub = 0; sub < S; ++sub)
+            umma_bf16(d_tmem + static_cast<uint32_t>(sub) * n_stride, a_kh + sub * sub_step + 2u * k,
+                      b_st + 2u * k, idesc, accumulate);
+        }
+      };
+      auto release_b = [&]() {
+        umma_commit(empty_b0 + sb * 8u);
+        if (++sb == static_cast<uint32_t>(p.stages_b)) {
+          sb = 0;
+          pb ^= 1u;
+        }
+      };
+      if (g < p.groups_main) {
 #pragma unroll
         for (int kh = 0; kh < KHT; ++kh) {
-          const uint32_t accumulate = (kb | k | kh) != 0 ? 1u : 0u;
-          const uint64_t b_k = b_st + kh * kh_step_b + 2u * k;
-#pragma unroll
-          for (int sub = 0; sub < S; ++sub) {
-            const uint64_t a_k = a_st + sub * sub_step + kh * kh_step_a + 2u * k;
-            const uint32_t d_sub = d_tmem + static_cast<uint32_t>(sub) * bn;
-            umma_bf16(d_sub, a_k, b_k, idesc, accumulate);
-            if (HALVES == 2) umma_bf16(d_sub + 256u, a_k, b_k + 2048u, idesc, accumulate);
+          if (kh % BT == 0) {
+            if (!mma_wait(full_b0 + sb * 8u, pb, s, p)) {
+              aborted = true;
+              break;
+            }
+            tc_fence_after();
           }
+          issue(kh, kh % BT);
+          if (kh % BT == BT - 1) release_b();
+        }
+      } else {
+        // second segment: one weight tile, A without halo
+        if (!mma_wait(full_b0 + sb * 8u, pb, s, p)) {
+          aborted = true;
+        } else {
+          tc_fence_after();
+          issue(0, 0);
+          release_b();
         }
       }
-      umma_commit(empty0 + st * 8u);
-      if (++st == static_cast<uint32_t>(p.stages)) {
-        st = 0;
-        ph ^= 1u;
+      if (aborted) break;
+      if (!COMBINED) {
+        umma_commit(empty_a0 + sa * 8u);
+        if (++sa == static_cast<uint32_t>(p.stages_a)) {
+          sa = 0;
+          pa ^= 1u;
+        }
       }
     }
     if (aborted) break;
@@ -490,14 +558,33 @@ __device__ __forceinline__ void lane_emit(const ConvParams& p, const Smem& s, ui
   }
 }
 
+// Column taps in N (nw = 3): the lane holds, for its computed column c, the
+// partial sums P_u (u = 0, 1, 2: BN columns each) of column tap u over the
+// input column at c.  Output column c needs P_0 from column c - 1, P_1 from
+// c and P_2 from c + 1: the neighbouring lanes of the same tile row (a warp
+// holds two rows of 16; the edge columns 0 and 15 are halo and not output).
+template <int NB>
+__device__ __noinline__ void lane_emit_taps_in_n(const ConvParams& p, const Smem& s,
+                                                    uint32_t taddr, int n0, bool valid,
+                                                    size_t vox, const TileCoord& tc, int h,
+                                                    int w) {
+  float v[NB], t[NB];
+  tmem_load_chunk<NB>(taddr + NB, v);
+  tmem_load_chunk<NB>(taddr, t);
+#pragma unroll
+  for (int j = 0; j < NB; ++j) v[j] += __shfl_up_sync(0xffffffffu, t[j], 1);
+  tmem_load_chunk<NB>(taddr + 2 * NB, t);
+#pragma unroll
+  for (int j = 0; j < NB; ++j) v[j] += __shfl_down_sync(0xffffffffu, t[j], 1) + s.bias[n0 + j];
+  if (valid) emit_chunk<NB>(p, 0, n0, tc, h, w, vox, v);
+}
+
 __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base, int warp,
                          int lane, int crank) {
   const int q = warp & 3;           // TMEM lane quarter this warp may access
   const int grp = (warp - 2) >> 2;  // epilogue group 0 or 1
   const int row = q * 32 + lane;
   const float rootC = sqrtf(static_cast<float>(p.cout));
-  const bool split_cols = p.S == 1;
-  const int half = p.BN / 2;
   uint32_t ti = 0;
   for (int tile = tile_first(p); tile < p.num_tiles; tile += tile_stride(p), ++ti) {
     const uint32_t acc = ti % p.num_acc;
@@ -514,25 +601,26 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
     tc_fence_after();
     const TileCoord tc = decode_tile(p, tile, crank);
     const int n0 = tc.n_tile * p.BN;
-    for (int sub = split_cols ? 0 : grp; sub < p.S; sub += split_cols ? 1 : 2) {
-      const int idx = sub * kBM + row;  // voxel of the tile, row-major
+    for (int sub = grp; sub < p.S; sub += 2) {  // the groups take alternate sub-tiles
+      const int idx = sub * kBM + row;  // computed voxel of the tile, row-major
+      const int c = idx % p.tile_cols;
       const int h = tc.th * p.tile_rows + idx / p.tile_cols;
-      const int w = tc.tw * p.tile_cols + idx % p.tile_cols;
-      const bool valid = h < p.H && w < p.W;
+      const int w = tc.tw * p.out_cols + c - (p.nw > 1 ? 1 : 0);
+      const bool valid = h < p.H && w < p.W && (p.nw == 1 || (c >= 1 && c <= p.tile_cols - 2));
       // output voxel: (t, h, w), or (t, 2h + p', 2w + q') of the 2H x 2W output in phase mode
       const size_t vox = p.phases == 4
                              ? (static_cast<size_t>(tc.t) * 2 * p.H + 2 * h + (tc.phase >> 1)) *
                                        (2 * p.W) + 2 * w + (tc.phase & 1)
                              : (static_cast<size_t>(tc.t) * p.H + h) * p.W + w;
+      const uint32_t n_stride = conv_tc_acc_stride(p);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                             acc * static_cast<uint32_t>(p.S * p.BN) +
-                             static_cast<uint32_t>(sub * p.BN);
-      const int c_lo = split_cols ? grp * half : 0;
-      const int c_hi = split_cols ? c_lo + half : p.BN;
-      if (p.ep.act == nullptr) {
-        lane_emit(p, s, taddr, c_lo, c_hi, n0, valid, vox, tc, h, w);
+                             (acc * static_cast<uint32_t>(p.S) + static_cast<uint32_t>(sub)) * n_stride;
+      if (p.nw > 1) {
+        lane_emit_taps_in_n<16>(p, s, taddr, n0, valid, vox, tc, h, w);  // BN = 16
+      } else if (p.ep.act == nullptr) {
+        lane_emit(p, s, taddr, 0, p.BN, n0, valid, vox, tc, h, w);
       } else {
-        float ss = lane_pass1(p, s, taddr, c_lo, c_hi, n0, valid, vox);
+        float ss = lane_pass1(p, s, taddr, 0, p.BN, n0, valid, vox);
         if (p.nsplit == 2) {
           // the other half of the channels is in the peer CTA: swap partial sums
           const int slot = (ti & 1u) * 256 + sub * 128 + row;
@@ -549,24 +637,9 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
           if (!got) return;
           __syncwarp();
           ss += s.xpart[slot];
-        } else if (split_cols) {
-          // exchange the two halves' sums through shared memory (bounded wait)
-          float* part = s.ss_part + (ti & 1u) * 256;
-          part[grp * 128 + row] = ss;
-          mbar_arrive(smem_u32(s.ssbar));
-          int got = 0;
-          if (lane == 0)
-            got = mbar_wait_bounded(smem_u32(s.ssbar), ti & 1u, s.abort_flag, p.err,
-                                    DEVERR_TIMEOUT_EPILOGUE)
-                      ? 1
-                      : 0;
-          got = __shfl_sync(0xffffffffu, got, 0);
-          if (!got) return;
-          __syncwarp();
-          ss += part[(grp ^ 1) * 128 + row];
         }
         const float rs = rootC / fmaxf(sqrtf(ss), p.ep.eps);
-        lane_pass2(p, s, taddr, c_lo, c_hi, n0, valid, vox, rs);
+        lane_pass2(p, s, taddr, 0, p.BN, n0, valid, vox, rs);
       }
     }
     tc_fence_before();
@@ -580,16 +653,19 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < p.stages; ++i) {
-      mbar_init(smem_u32(&s.full[i]), 1);
-      mbar_init(smem_u32(&s.empty[i]), 1);
+    for (int i = 0; i < p.stages_a; ++i) {
+      mbar_init(smem_u32(&s.full_a[i]), 1);
+      mbar_init(smem_u32(&s.empty_a[i]), 1);
+    }
+    for (int i = 0; i < p.stages_b; ++i) {
+      mbar_init(smem_u32(&s.full_b[i]), 1);
+      mbar_init(smem_u32(&s.empty_b[i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&s.tfull[i]), 1);
       mbar_init(smem_u32(&s.tempty[i]), 256);
     }
     mbar_init(smem_u32(s.drain), 1);
-    mbar_init(smem_u32(s.ssbar), 256);
     mbar_init(smem_u32(&s.xbar[0]), 256);  // 256 epilogue threads of the peer CTA
     mbar_init(smem_u32(&s.xbar[1]), 256);
     *s.abort_flag = 0;
@@ -625,16 +701,16 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
     if (lane == 0) producer(p, s, crank);
   } else if (warp == 1) {
     if (lane == 0) {
-      if (p.rowhalo)
-        mma_issuer<2, 1, 3>(p, s, tmem_base);
-      else if (p.BN > 256)
-        mma_issuer<1, 2, 1>(p, s, tmem_base);
-      else if (p.S == 1)
-        mma_issuer<1, 1, 1>(p, s, tmem_base);
-      else if (p.S == 2)
-        mma_issuer<2, 1, 1>(p, s, tmem_base);
+      // S = 2 throughout; narrow layers (and 1-row kernels) put a group's
+      // window and weight tiles in one stage
+      if (p.kh_eff == 1)
+        mma_issuer<2, 1, 1, true>(p, s, tmem_base);
+      else if (p.kh_eff == 2)
+        p.combined ? mma_issuer<2, 2, 2, true>(p, s, tmem_base)
+                   : mma_issuer<2, 2, 1, false>(p, s, tmem_base);
       else
-        mma_issuer<4, 1, 1>(p, s, tmem_base);
+        p.combined ? mma_issuer<2, 3, 3, true>(p, s, tmem_base)
+                   : mma_issuer<2, 3, 1, false>(p, s, tmem_base);
     }
   } else {
     epilogue(p, s, tmem_base, warp, lane, crank);
@@ -653,23 +729,35 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
 
 }  // namespace
 
-size_t conv_tc_smem_bytes(const ConvParams& p, int stages) {
-  const size_t stage = static_cast<size_t>(conv_tc_a_bytes(p)) + conv_tc_b_bytes(p);
-  return 1024 + stages * stage + kCtrlBytes;
+size_t conv_tc_smem_bytes(const ConvParams& p) {
+  return 1024 + static_cast<size_t>(p.stages_a) * conv_tc_a_bytes(p) +
+         static_cast<size_t>(p.stages_b) * conv_tc_b_bytes(p) + kCtrlBytes;
 }
 
-int conv_tc_stages_for(const ConvParams& p) {
-  const size_t limit = 232448;  // 227 KB opt-in dynamic shared memory per block
-  int st = kMaxStages;
-  while (st > 2 && conv_tc_smem_bytes(p, st) > limit) --st;
-  return st;
+void conv_tc_choose_stages(ConvParams& p) {
+  const size_t budget = 232448 - 1024 - kCtrlBytes;  // 227 KB opt-in per block
+  const size_t a = conv_tc_a_bytes(p), b = conv_tc_b_bytes(p);
+  if (p.combined) {
+    // one stage per group: equal depths
+    size_t n = budget / (a + b);
+    if (n > static_cast<size_t>(kMaxStages)) n = kMaxStages;
+    p.stages_a = p.stages_b = static_cast<int>(n < 2 ? 2 : n);
+    return;
+  }
+  // each A window serves kh_eff weight tiles: two A stages, the rest for B
+  size_t nb = (budget - 2 * a) / b;
+  if (nb > static_cast<size_t>(kMaxStages)) nb = kMaxStages;
+  p.stages_b = static_cast<int>(nb < 2 ? 2 : nb);
+  size_t na = (budget - p.stages_b * b) / a;
+  if (na > 4) na = 4;
+  p.stages_a = static_cast<int>(na < 2 ? 2 : na);
 }
 
 namespace {
 size_t launch_smem(const ConvParams& p) {
   // Every CTA allocates all 512 TMEM columns, so exactly one may live on an SM:
   // ask for more than half of the SM's shared memory even when the ring is small.
-  size_t smem = conv_tc_smem_bytes(p, p.stages);
+  size_t smem = conv_tc_smem_bytes(p);
   if (smem < 120 * 1024) smem = 120 * 1024;
   return smem;
 }

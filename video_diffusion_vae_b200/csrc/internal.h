@@ -54,28 +54,41 @@ struct ConvParams {
   int BN, n_tiles;
   int S;             // MMA sub-tiles per CTA tile; S * BN <= 512 TMEM columns
   int tile_rows, tile_cols;  // CTA tile, tile_rows * tile_cols = 128 S voxels of one frame
-  int tile_cols_log2;
-  int rowhalo;       // 1: a K block is (kt, kw, 64 channels) with all KH row taps inside:
-                     //    one A box of tile_rows + KH - 1 rows, KH weight tiles; the row
-                     //    tap selects a row offset of the A operand (small BN only)
+  int kh_eff, kw_eff;  // row / column taps per A window: KH, KW (2, 2 in phase mode; kw_eff
+                       // = 1 when the column taps ride in N)
+  int nw;            // column taps per MMA: 1, or KW (narrow layers: N = KW * BN, the
+                     // epilogue adds the taps' partial sums from the neighbouring columns)
+  int out_cols;      // output columns per tile: tile_cols, or tile_cols - 2 when nw = KW
+  int b_tiles;       // weight tiles per B-ring stage: 1, or kh_eff (a group's row taps
+                     // behind one wait, for narrow BN where one tile is little MMA work)
+  int combined;      // 1 (b_tiles == kh_eff): a group's A window and weight tiles travel
+                     // in one stage on one barrier (A and B rings in lockstep)
   int tiles_w, tiles_h, m_tiles, num_tiles;
-  int stages, num_acc;
-  int kblocks_main, kblocks;
+  int stages_a, stages_b, num_acc;  // A-window ring, weight-tile ring, TMEM accumulators
+  int groups_main;   // K groups of the main segment: (kt, column tap, 64 input channels)
+  int groups;        // + one group per 64 channels of the second segment
   ConvEpilogue ep;
   unsigned* err;
 };
 
-// Shared-memory bytes of one ring stage's A part (1024-aligned) and B part.
+// A window of a main-segment K group: the tile's rows plus the row-tap halo.
+__host__ __device__ inline uint32_t conv_tc_a_rows(const ConvParams& p) {
+  return static_cast<uint32_t>(p.tile_rows + p.kh_eff - 1);
+}
+// Shared-memory bytes of one A-ring stage (1024-aligned) and one B-ring stage.
 __host__ __device__ inline uint32_t conv_tc_a_bytes(const ConvParams& p) {
-  const uint32_t rows = p.rowhalo ? static_cast<uint32_t>(p.tile_rows + p.KH - 1)
-                                  : static_cast<uint32_t>(p.tile_rows);
-  return (rows * static_cast<uint32_t>(p.tile_cols) * 128u + 1023u) & ~1023u;
+  return (conv_tc_a_rows(p) * static_cast<uint32_t>(p.tile_cols) * 128u + 1023u) & ~1023u;
 }
 __host__ __device__ inline uint32_t conv_tc_b_bytes(const ConvParams& p) {
-  return static_cast<uint32_t>(p.rowhalo ? p.KH : 1) * static_cast<uint32_t>(p.BN) * 128u;
+  return static_cast<uint32_t>(p.b_tiles * p.nw * p.BN) * 128u;
 }
-size_t conv_tc_smem_bytes(const ConvParams& p, int stages);
-int conv_tc_stages_for(const ConvParams& p);
+// TMEM columns per sub-tile accumulator: the MMA's N (nw BN) rounded up to 32.
+__host__ __device__ inline uint32_t conv_tc_acc_stride(const ConvParams& p) {
+  return (static_cast<uint32_t>(p.nw * p.BN) + 31u) & ~31u;
+}
+size_t conv_tc_smem_bytes(const ConvParams& p);
+// Sets p.stages_a / p.stages_b for the layer (needs BN, tile shape, kh_eff).
+void conv_tc_choose_stages(ConvParams& p);
 // Clusters of 2 that fit on the device at once (nsplit = 2 launches), 0 on error.
 int conv_tc_max_clusters(const ConvParams& p);
 cudaError_t launch_conv_tc(const ConvParams& p, int grid, cudaStream_t stream);
