@@ -108,7 +108,9 @@ struct TileCoord {
 };
 
 // Tile order: N tile fastest, then upsample phase (the four phases of an M
-// tile read the same input), then M tiles (column, row, frame).
+// tile read the same input), then frame (the KT temporal taps of neighbouring
+// frames read the same input frames: a frame of a large layer does not stay
+// in L2 until the next frame's tiles come round), then tile column and row.
 // With nsplit = 2 the two CTAs of a cluster take the same tiles and the CTA
 // rank is the N tile.
 __device__ __forceinline__ TileCoord decode_tile(const ConvParams& p, int tile, int crank) {
@@ -123,10 +125,10 @@ __device__ __forceinline__ TileCoord decode_tile(const ConvParams& p, int tile, 
   }
   c.phase = m % p.phases;
   m /= p.phases;
+  c.t = m % p.T;
+  m /= p.T;
   c.tw = m % p.tiles_w;
-  m /= p.tiles_w;
-  c.th = m % p.tiles_h;
-  c.t = m / p.tiles_h;
+  c.th = m / p.tiles_w;
   return c;
 }
 
