@@ -461,12 +461,23 @@ __device__ __forceinline__ void store_raw(const ConvParams& p, int c0, int n0, s
 template <int NC>
 __device__ __forceinline__ void store_act(const ConvParams& p, const Smem& s, int c0, int n0,
                                           size_t ovox, float rs, const float (&v)[NC]) {
-  float a[NC];
+  // packed pairs: SiLU_half((v rs) gamma/2 + beta/2)
+  const float2 r2 = make_float2(rs, rs);
+  const float2* g2 = reinterpret_cast<const float2*>(s.gamma + n0 + c0);
+  const float2* b2 = reinterpret_cast<const float2*>(s.beta + n0 + c0);
+  uint4* d = reinterpret_cast<uint4*>(p.ep.act + ovox * p.cout + n0 + c0);
 #pragma unroll
-  for (int j = 0; j < NC; ++j) {
-    a[j] = silu_half(v[j] * rs * s.gamma[n0 + c0 + j] + s.beta[n0 + c0 + j]);
+  for (int q = 0; q < NC / 8; ++q) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 8 * q + 2 * e;
+      const float2 o =
+          silu_half2(ffma2(fmul2(make_float2(v[j], v[j + 1]), r2), g2[j / 2], b2[j / 2]));
+      w[e] = pack_bf16x2(o.x, o.y);
+    }
+    d[q] = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  store_bf16<NC>(p.ep.act + ovox * p.cout + n0 + c0, a);
 }
 
 // Outputs that need no RMS statistic: the raw result and the video.
@@ -511,8 +522,14 @@ __device__ __forceinline__ void pass1_chunk(const ConvParams& p, const Smem& s, 
                                             int c0, int n0, bool valid, size_t vox, float& ss) {
   float v[NC];
   result_chunk<NC>(p, s, taddr, c0, n0, valid, vox, v);
+  float2 sa = make_float2(0.0f, 0.0f), sb = sa;  // two packed chains
 #pragma unroll
-  for (int j = 0; j < NC; ++j) ss = fmaf(v[j], v[j], ss);
+  for (int j = 0; j < NC; j += 4) {
+    const float2 x0 = make_float2(v[j], v[j + 1]), x1 = make_float2(v[j + 2], v[j + 3]);
+    sa = ffma2(x0, x0, sa);
+    sb = ffma2(x1, x1, sb);
+  }
+  ss += (sa.x + sa.y) + (sb.x + sb.y);
   if (valid) store_raw<NC>(p, c0, n0, vox, v);
   tmem_store_chunk<NC>(taddr + c0, v);
 }

@@ -187,14 +187,19 @@ __global__ void __launch_bounds__(kRingThreads, 1)
   const int cw = warp - 1;
   const int sub = lane % L, grp = lane / L, gpw = 32 / L;
   const int nvec = C / 8;
-  float g[CH][8], b[CH][8];
+  // channel pairs (2e, 2e + 1) of each of the lane's vectors, pre-halved
+  float2 g[CH][4], b[CH][4];
 #pragma unroll
   for (int k = 0; k < CH; ++k) {
     const int vi = sub + k * L;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      g[k][e] = vi < nvec ? 0.5f * __ldg(gamma + vi * 8 + e) : 0.0f;
-      b[k][e] = vi < nvec ? 0.5f * __ldg(beta + vi * 8 + e) : 0.0f;
+    for (int e = 0; e < 4; ++e) {
+      g[k][e] = vi < nvec ? make_float2(0.5f * __ldg(gamma + vi * 8 + 2 * e),
+                                        0.5f * __ldg(gamma + vi * 8 + 2 * e + 1))
+                          : make_float2(0.0f, 0.0f);
+      b[k][e] = vi < nvec ? make_float2(0.5f * __ldg(beta + vi * 8 + 2 * e),
+                                        0.5f * __ldg(beta + vi * 8 + 2 * e + 1))
+                          : make_float2(0.0f, 0.0f);
     }
   }
   const float rootC = sqrtf(static_cast<float>(C));
@@ -218,31 +223,39 @@ __global__ void __launch_bounds__(kRingThreads, 1)
       const bool live = vl < nv;
       const uint4* src = reinterpret_cast<const uint4*>(stage + static_cast<size_t>(vl) * C * 2);
       uint4 raw[CH];
-      float ss = 0.0f;
+      float2 ssa = make_float2(0.0f, 0.0f), ssb = ssa;  // two packed chains
 #pragma unroll
       for (int k = 0; k < CH; ++k) {
         const int vi = sub + k * L;
         raw[k] = (live && vi < nvec) ? src[vi] : make_uint4(0u, 0u, 0u, 0u);
         float v[8];
         unpack<8>(raw[k], v);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
+        const float2 p0 = make_float2(v[0], v[1]), p1 = make_float2(v[2], v[3]);
+        const float2 p2 = make_float2(v[4], v[5]), p3 = make_float2(v[6], v[7]);
+        ssa = ffma2(p0, p0, ssa);
+        ssb = ffma2(p1, p1, ssb);
+        ssa = ffma2(p2, p2, ssa);
+        ssb = ffma2(p3, p3, ssb);
       }
+      float ss = (ssa.x + ssa.y) + (ssb.x + ssb.y);
       for (int off = L >> 1; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
       const float r = rootC / fmaxf(sqrtf(ss), eps);
+      const float2 r2 = make_float2(r, r);
       uint4* dst = reinterpret_cast<uint4*>(y + (v0 + vl) * C);
 #pragma unroll
       for (int k = 0; k < CH; ++k) {
         const int vi = sub + k * L;
         if (!live || vi >= nvec) continue;
-        float v[8], o[8];
+        float v[8];
         unpack<8>(raw[k], v);
+        uint32_t w4[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = silu_half(fmaf(v[e], r * g[k][e], b[k][e]));
-        uint4 w;
-        w.x = pack_bf16x2(o[0], o[1]); w.y = pack_bf16x2(o[2], o[3]);
-        w.z = pack_bf16x2(o[4], o[5]); w.w = pack_bf16x2(o[6], o[7]);
-        dst[vi] = w;
+        for (int e = 0; e < 4; ++e) {
+          const float2 o = silu_half2(ffma2(make_float2(v[2 * e], v[2 * e + 1]),
+                                            fmul2(r2, g[k][e]), b[k][e]));
+          w4[e] = pack_bf16x2(o.x, o.y);
+        }
+        dst[vi] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
     }
     __syncwarp();

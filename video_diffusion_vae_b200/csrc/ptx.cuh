@@ -284,6 +284,30 @@ __device__ __forceinline__ float tanh_approx(float x) {
 // operation per element.  Callers fold the 1/2 into the affine coefficients.
 __device__ __forceinline__ float silu_half(float h) { return fmaf(h, tanh_approx(h), h); }
 __device__ __forceinline__ float silu_fast(float s) { return silu_half(0.5f * s); }
+// Packed two-lane fp32 arithmetic (sm_100 f32x2: one instruction for both
+// lanes, each rounded as the scalar operation would be).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+// silu_half on a pair: h + h tanh(h).
+__device__ __forceinline__ float2 silu_half2(float2 h) {
+  return ffma2(h, make_float2(tanh_approx(h.x), tanh_approx(h.y)), h);
+}
 // Non-tensor bulk copy global -> shared memory (16-byte aligned addresses, size
 // a multiple of 16), completing `bytes` of transaction count on `bar`.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
