@@ -111,3 +111,25 @@ def test_conv_wide_tiles_sampled():
     assert_close(got, ref, torch.bfloat16, "wide tiles sampled")
     assert torch.isfinite(yc).all()
     assert B.device_error() == 0
+
+
+def test_conv_epilogue_16_byte_aligned_buffers():
+    """Output and residual 16- but not 32-byte aligned take the 128-bit
+    epilogue accesses; the result is identical to the 256-bit path's."""
+    T, H, W, cin, cout = 2, 9, 20, 64, 128
+    x, w, b = synth.conv_input(cin=cin, cout=cout, T=T, H=H, W=W, seed=21)
+    res = torch.randn(cout, T, H, W, generator=torch.Generator().manual_seed(22)).bfloat16().float()
+    pk = B.prepack_conv(w.cuda().bfloat16(), b.cuda())
+    xd, rd = to_cl(x), to_cl(res)
+    y32 = B.causal_conv3d(xd, pk, residual=rd)
+    n = T * H * W * cout
+    obuf = torch.empty(n + 8, dtype=torch.bfloat16, device="cuda")
+    rbuf = torch.empty(n + 8, dtype=torch.bfloat16, device="cuda")
+    out16 = obuf[8:].view(T, H, W, cout)    # 16 bytes past a 256-byte boundary
+    res16 = rbuf[8:].view(T, H, W, cout)
+    res16.copy_(rd)
+    assert out16.data_ptr() % 32 == 16 and res16.data_ptr() % 32 == 16
+    B.causal_conv3d(xd, pk, residual=res16, out=out16)
+    torch.cuda.synchronize()
+    assert torch.equal(out16, y32)
+    assert_close(from_cl(y32), O.causal_conv3d(x, w, b) + res.double().numpy(), torch.bfloat16, "res")

@@ -237,6 +237,9 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
     a.ep.bias2 = reinterpret_cast<const float*>(static_cast<const char*>(a.packed2) + L2.bias_off);
   }
   p.ep = a.ep;
+  // 256-bit epilogue accesses need 32-byte aligned rows and bases
+  auto a32 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 31u) == 0; };
+  p.ep.vec32 = (a.cout % 16 == 0 && a32(a.ep.residual) && a32(a.ep.out) && a32(a.ep.act)) ? 1 : 0;
   p.err = d.err;
   const int box_rows = p.BN;  // BN <= 256
   const int a_rows = static_cast<int>(conv_tc_a_rows(p));

@@ -383,6 +383,31 @@ __device__ __forceinline__ void tmem_load_chunk<16>(uint32_t taddr, float (&v)[1
 
 template <int NC>
 __device__ __forceinline__ void add_residual(const ConvEpilogue& ep, size_t off, float (&v)[NC]) {
+  if (ep.vec32) {
+    if (ep.residual_f32) {
+      const float* r = static_cast<const float*>(ep.residual) + off;
+#pragma unroll
+      for (int q = 0; q < NC / 8; ++q) {
+        uint32_t u[8];
+        ld_global_v8(r + 8 * q, u);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[8 * q + e] += __uint_as_float(u[e]);
+      }
+    } else {
+      const __nv_bfloat16* r = static_cast<const __nv_bfloat16*>(ep.residual) + off;
+#pragma unroll
+      for (int q = 0; q < NC / 16; ++q) {
+        uint32_t u[8];
+        ld_global_v8(r + 16 * q, u);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          v[16 * q + 2 * e] += bf16lo(u[e]);
+          v[16 * q + 2 * e + 1] += bf16hi(u[e]);
+        }
+      }
+    }
+    return;
+  }
   if (ep.residual_f32) {
     const float4* r = reinterpret_cast<const float4*>(static_cast<const float*>(ep.residual) + off);
 #pragma unroll
@@ -412,7 +437,17 @@ __device__ __forceinline__ void add_residual(const ConvEpilogue& ep, size_t off,
 }
 
 template <int NC>
-__device__ __forceinline__ void store_bf16(__nv_bfloat16* dst, const float (&v)[NC]) {
+__device__ __forceinline__ void store_bf16(__nv_bfloat16* dst, const float (&v)[NC], bool vec32) {
+  if (vec32) {
+#pragma unroll
+    for (int q = 0; q < NC / 16; ++q) {
+      uint32_t u[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) u[e] = pack_bf16x2(v[16 * q + 2 * e], v[16 * q + 2 * e + 1]);
+      st_global_v8(dst + 16 * q, u);
+    }
+    return;
+  }
   uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
   for (int q = 0; q < NC / 8; ++q) {
@@ -426,7 +461,17 @@ __device__ __forceinline__ void store_bf16(__nv_bfloat16* dst, const float (&v)[
 }
 
 template <int NC>
-__device__ __forceinline__ void store_f32(float* dst, const float (&v)[NC]) {
+__device__ __forceinline__ void store_f32(float* dst, const float (&v)[NC], bool vec32) {
+  if (vec32) {
+#pragma unroll
+    for (int q = 0; q < NC / 8; ++q) {
+      uint32_t u[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) u[e] = __float_as_uint(v[8 * q + e]);
+      st_global_v8(dst + 8 * q, u);
+    }
+    return;
+  }
   float4* d = reinterpret_cast<float4*>(dst);
 #pragma unroll
   for (int q = 0; q < NC / 4; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
@@ -452,9 +497,9 @@ __device__ __forceinline__ void store_raw(const ConvParams& p, int c0, int n0, s
   if (ep.out != nullptr) {
     const size_t off = ovox * p.cout + n0 + c0;
     if (ep.out_f32)
-      store_f32<NC>(static_cast<float*>(ep.out) + off, v);
+      store_f32<NC>(static_cast<float*>(ep.out) + off, v, ep.vec32 != 0);
     else
-      store_bf16<NC>(static_cast<__nv_bfloat16*>(ep.out) + off, v);
+      store_bf16<NC>(static_cast<__nv_bfloat16*>(ep.out) + off, v, ep.vec32 != 0);
   }
 }
 
@@ -465,7 +510,23 @@ __device__ __forceinline__ void store_act(const ConvParams& p, const Smem& s, in
   const float2 r2 = make_float2(rs, rs);
   const float2* g2 = reinterpret_cast<const float2*>(s.gamma + n0 + c0);
   const float2* b2 = reinterpret_cast<const float2*>(s.beta + n0 + c0);
-  uint4* d = reinterpret_cast<uint4*>(p.ep.act + ovox * p.cout + n0 + c0);
+  __nv_bfloat16* dst = p.ep.act + ovox * p.cout + n0 + c0;
+  if (p.ep.vec32) {
+#pragma unroll
+    for (int q = 0; q < NC / 16; ++q) {
+      uint32_t w[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int j = 16 * q + 2 * e;
+        const float2 o =
+            silu_half2(ffma2(fmul2(make_float2(v[j], v[j + 1]), r2), g2[j / 2], b2[j / 2]));
+        w[e] = pack_bf16x2(o.x, o.y);
+      }
+      st_global_v8(dst + 16 * q, w);
+    }
+    return;
+  }
+  uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
   for (int q = 0; q < NC / 8; ++q) {
     uint32_t w[4];

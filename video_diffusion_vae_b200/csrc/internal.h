@@ -35,6 +35,7 @@ struct ConvEpilogue {
   const float* beta;        // fp32 [cout] for act
   float eps;
   __nv_bfloat16* video;     // 2x2 pixel-shuffled NCDHW [cout/4][T][2H][2W], or null
+  int vec32;                // residual / out / act are 32-byte aligned: 256-bit accesses
 };
 
 struct ConvParams {

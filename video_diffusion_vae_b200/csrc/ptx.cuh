@@ -284,6 +284,20 @@ __device__ __forceinline__ float tanh_approx(float x) {
 // operation per element.  Callers fold the 1/2 into the affine coefficients.
 __device__ __forceinline__ float silu_half(float h) { return fmaf(h, tanh_approx(h), h); }
 __device__ __forceinline__ float silu_fast(float s) { return silu_half(0.5f * s); }
+// 32-byte global accesses (sm_100 256-bit vectors): one full sector per thread.
+// The address must be 32-byte aligned.
+__device__ __forceinline__ void ld_global_v8(const void* p, uint32_t (&r)[8]) {
+  asm volatile("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "l"(p));
+}
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&r)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 // Packed two-lane fp32 arithmetic (sm_100 f32x2: one instruction for both
 // lanes, each rounded as the scalar operation would be).
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
