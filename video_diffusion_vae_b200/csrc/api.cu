@@ -254,6 +254,10 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
     if (!encode_act(&p.tmA2, a.x2, a.cin2_pad, a.W, a.H, a.T, p.tile_cols, p.tile_rows)) return WVAE_ERR_CUDA;
     if (!encode_weights(&p.tmB2, a.packed2, a.cin2_pad, L.cout_pad, box_rows)) return WVAE_ERR_CUDA;
   }
+  p.early_release = (p.num_acc == 1 && a.ep.act != nullptr && a.ep.out != nullptr &&
+                     a.ep.out_f32 && p.num_tiles > slots)
+                        ? 1
+                        : 0;
   int grid;
   if (p.nsplit == 2) {
     int clusters = conv_tc_max_clusters(p);

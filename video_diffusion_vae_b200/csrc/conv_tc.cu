@@ -580,7 +580,8 @@ __device__ __forceinline__ void tmem_store_chunk(uint32_t taddr, const float (&v
 // bias again), and into the returned sum of squares.
 template <int NC>
 __device__ __forceinline__ void pass1_chunk(const ConvParams& p, const Smem& s, uint32_t taddr,
-                                            int c0, int n0, bool valid, size_t vox, float& ss) {
+                                            int c0, int n0, bool valid, size_t vox, float& ss,
+                                            bool keep) {
   float v[NC];
   result_chunk<NC>(p, s, taddr, c0, n0, valid, vox, v);
   float2 sa = make_float2(0.0f, 0.0f), sb = sa;  // two packed chains
@@ -592,16 +593,64 @@ __device__ __forceinline__ void pass1_chunk(const ConvParams& p, const Smem& s, 
   }
   ss += (sa.x + sa.y) + (sb.x + sb.y);
   if (valid) store_raw<NC>(p, c0, n0, vox, v);
-  tmem_store_chunk<NC>(taddr + c0, v);
+  if (keep) tmem_store_chunk<NC>(taddr + c0, v);
 }
+// keep = false: h is not stored back (the caller re-reads it from the fp32
+// raw output instead).
 __device__ __forceinline__ float lane_pass1(const ConvParams& p, const Smem& s, uint32_t taddr,
-                                           int c_lo, int c_hi, int n0, bool valid, size_t vox) {
+                                           int c_lo, int c_hi, int n0, bool valid, size_t vox,
+                                           bool keep) {
   float ss = 0.0f;
   int c0 = c_lo;
-  for (; c0 + 32 <= c_hi; c0 += 32) pass1_chunk<32>(p, s, taddr, c0, n0, valid, vox, ss);
-  if (c0 < c_hi) pass1_chunk<16>(p, s, taddr, c0, n0, valid, vox, ss);
-  tmem_wait_st();
+  for (; c0 + 32 <= c_hi; c0 += 32) pass1_chunk<32>(p, s, taddr, c0, n0, valid, vox, ss, keep);
+  if (c0 < c_hi) pass1_chunk<16>(p, s, taddr, c0, n0, valid, vox, ss, keep);
+  if (keep) tmem_wait_st();
   return ss;
+}
+
+// Second pass reading h back from the fp32 raw output this thread wrote in
+// pass 1 (the accumulator is released already).
+__device__ __forceinline__ void lane_pass2_global(const ConvParams& p, const Smem& s, int n0,
+                                                 bool valid, size_t vox, float rs) {
+  if (!valid) return;
+  const float* h = static_cast<const float*>(p.ep.out) + vox * p.cout + n0;
+  int c0 = 0;
+  for (; c0 + 32 <= p.BN; c0 += 32) {
+    float v[32];
+    if (p.ep.vec32) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t u[8];
+        ld_global_v8(h + c0 + 8 * q, u);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[8 * q + e] = __uint_as_float(u[e]);
+      }
+    } else {
+      const float4* h4 = reinterpret_cast<const float4*>(h + c0);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 f = h4[q];
+        v[4 * q] = f.x;
+        v[4 * q + 1] = f.y;
+        v[4 * q + 2] = f.z;
+        v[4 * q + 3] = f.w;
+      }
+    }
+    store_act<32>(p, s, c0, n0, vox, rs, v);
+  }
+  if (c0 < p.BN) {
+    float v[16];
+    const float4* h4 = reinterpret_cast<const float4*>(h + c0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 f = h4[q];
+      v[4 * q] = f.x;
+      v[4 * q + 1] = f.y;
+      v[4 * q + 2] = f.z;
+      v[4 * q + 3] = f.w;
+    }
+    store_act<16>(p, s, c0, n0, vox, rs, v);
+  }
 }
 
 // Second pass: the next layer's activation SiLU(h r gamma + beta) from h in the lane.
@@ -665,6 +714,11 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
   const int grp = (warp - 2) >> 2;  // epilogue group 0 or 1
   const int row = q * 32 + lane;
   const float rootC = sqrtf(static_cast<float>(p.cout));
+  // With a fused norm and an fp32 raw output, pass 2 can read h back from that
+  // output, so the accumulator is released right after pass 1 and the next
+  // tile's main loop overlaps pass 2 (the host sets early_release where one
+  // accumulator fills TMEM and CTAs run several tiles).
+  const bool early = p.early_release != 0;
   uint32_t ti = 0;
   for (int tile = tile_first(p); tile < p.num_tiles; tile += tile_stride(p), ++ti) {
     const uint32_t acc = ti % p.num_acc;
@@ -700,7 +754,11 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
       } else if (p.ep.act == nullptr) {
         lane_emit(p, s, taddr, 0, p.BN, n0, valid, vox, tc, h, w);
       } else {
-        float ss = lane_pass1(p, s, taddr, 0, p.BN, n0, valid, vox);
+        float ss = lane_pass1(p, s, taddr, 0, p.BN, n0, valid, vox, !early);
+        if (early) {
+          tc_fence_before();
+          mbar_arrive(smem_u32(&s.tempty[acc]));
+        }
         if (p.nsplit == 2) {
           // the other half of the channels is in the peer CTA: swap partial sums
           const int slot = (ti & 1u) * 256 + sub * 128 + row;
@@ -719,11 +777,16 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
           ss += s.xpart[slot];
         }
         const float rs = rootC / fmaxf(sqrtf(ss), p.ep.eps);
-        lane_pass2(p, s, taddr, 0, p.BN, n0, valid, vox, rs);
+        if (early)
+          lane_pass2_global(p, s, n0, valid, vox, rs);
+        else
+          lane_pass2(p, s, taddr, 0, p.BN, n0, valid, vox, rs);
       }
     }
-    tc_fence_before();
-    mbar_arrive(smem_u32(&s.tempty[acc]));
+    if (!early) {
+      tc_fence_before();
+      mbar_arrive(smem_u32(&s.tempty[acc]));
+    }
   }
 }
 

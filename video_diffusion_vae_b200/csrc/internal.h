@@ -66,6 +66,8 @@ struct ConvParams {
                      // in one stage on one barrier (A and B rings in lockstep)
   int tiles_w, tiles_h, m_tiles, num_tiles;
   int stages_a, stages_b, num_acc;  // A-window ring, weight-tile ring, TMEM accumulators
+  int early_release; // 1: release the accumulator after epilogue pass 1 (fused norm + fp32
+                     //    raw output, one accumulator, several tiles per CTA)
   int groups_main;   // K groups of the main segment: (kt, column tap, 64 input channels)
   int groups;        // + one group per 64 channels of the second segment
   ConvEpilogue ep;
