@@ -424,26 +424,50 @@ def main():
     achieved_exec = conv_flops_exec / len(conv_idx) / (conv_launch_ms * 1e-3) / 1e12
     layer_ms = {layers[j][0]: statistics.mean(per_layer[i][j] for i in range(args.steps)) for j in range(nl)}
 
-    # ---- e2e: pinned host latents -> device, decode, video -> pinned host, per step
+    # ---- e2e: every step copies its latents from pinned host memory and its
+    # video back to pinned host memory; the copies run on a second stream,
+    # double-buffered, so step i's video leaves while step i+1 decodes (the
+    # way a serving loop runs).  No L2 flush here: a step's working set
+    # (~1.3 GB of activations) is ten times L2.
     zh = z[None].to(torch.bfloat16).contiguous().pin_memory()
-    vh = torch.empty(video.shape, dtype=torch.bfloat16).pin_memory()
-    for _ in range(2):
-        zd.copy_(zh, non_blocking=True)
-        step()
-        vh.copy_(video, non_blocking=True)
+    vh = [torch.empty(video.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    zdb = [zd, torch.empty_like(zd)]
+    vdb = [video, torch.empty_like(video)]
+    comp_s = torch.cuda.current_stream()
+    copy_s = torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event(enable_timing=False)  # noqa: E731
+    h2d_done, dec_done, d2h_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+
+    def e2e_steps(n):
+        for i in range(n):
+            b = i & 1
+            if i >= 2:
+                copy_s.wait_event(dec_done[b])      # step i-2 has read zdb[b]
+            with torch.cuda.stream(copy_s):
+                zdb[b].copy_(zh, non_blocking=True)
+                h2d_done[b].record(copy_s)
+            comp_s.wait_event(h2d_done[b])
+            if i >= 2:
+                comp_s.wait_event(d2h_done[b])      # step i-2's video has left vdb[b]
+            B.decode_trunk(zdb[b], tr, out=vdb[b], workspace=ws)
+            dec_done[b].record(comp_s)
+            copy_s.wait_event(dec_done[b])
+            with torch.cuda.stream(copy_s):
+                vh[b].copy_(vdb[b], non_blocking=True)
+                d2h_done[b].record(copy_s)
+
+    e2e_steps(3)
     torch.cuda.synchronize()
-    e2e_ms = []
-    for _ in range(args.steps):
-        flush.zero_()
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s.record()
-        zd.copy_(zh, non_blocking=True)
-        step()
-        vh.copy_(video, non_blocking=True)
-        e.record()
-        e.synchronize()
-        e2e_ms.append(s.elapsed_time(e))
-    e2e_value = throughput(T, args.steps, world, max_over_ranks(sum(e2e_ms), dev))
+    if world > 1:
+        dist.barrier()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(comp_s)
+    e2e_steps(args.steps)
+    copy_s.wait_stream(comp_s)
+    t_end.record(copy_s)
+    torch.cuda.synchronize()
+    e2e_value = throughput(T, args.steps, world, max_over_ranks(t_start.elapsed_time(t_end), dev))
+    assert torch.equal(vh[(args.steps - 1) & 1].cuda(), video)  # the copied-out result is the decode
 
     err = B.device_error()
     comp = None
@@ -484,7 +508,9 @@ def main():
                          "conv_share_of_step": conv_ms / statistics.mean(step_ms)},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": zh.numel() * 2,
-                    "d2h_bytes_per_step": vh.numel() * 2},
+                    "d2h_bytes_per_step": vh[0].numel() * 2,
+                    "copies": "pinned host <-> device on a second stream, double-buffered, "
+                              "overlapping the next step's decode; no L2 flush"},
             "gpu_launches": nl * args.steps,
             "clocks": clocks,
             "wall_s_timed_region": wall,

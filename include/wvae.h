@@ -80,6 +80,15 @@ WVAE_API int wvae_version(void);
  */
 WVAE_API wvae_status wvae_device_error(unsigned int* code, int reset);
 
+/* Self-test of the failure detection (the pages define no such call): enqueues
+ * one block whose thread waits on a pipeline barrier that nothing ever
+ * completes, with a limit of limit_us microseconds (1 .. 1,000,000) instead of
+ * the kernels' 2 s.  The wait gives up, records bit 0x10 in the error word and
+ * the kernel returns, so the context stays usable; read the outcome with
+ * wvae_device_error.  Returns WVAE_ERR_INVALID_ARG for a limit out of range,
+ * WVAE_ERR_NO_DEVICE / WVAE_ERR_CUDA as any launch. */
+WVAE_API wvae_status wvae_selftest_wait_timeout(unsigned int limit_us, wvae_stream_t stream);
+
 /* ---------------------------------------------------------------- norm-SiLU
  * Channel RMS-norm + affine + SiLU at every voxel v of x [T][H][W][C]:
  *   y[v,c] = SiLU( x[v,c] / max(||x[v,:]||_2, eps) * sqrt(C) * gamma[c] + beta[c] )

@@ -20,7 +20,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     declared = B.header_symbols()
-    assert len(declared) == 19
+    assert len(declared) == 20
     out = subprocess.check_output(["nm", "-D", "--defined-only", B.LIB_PATH], text=True)
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
     missing = [s for s in declared if s not in exported]
@@ -142,3 +142,10 @@ def test_binding_fails_loudly_without_library(tmp_path):
             mod.load(str(tmp_path / "missing.so"))
     finally:
         importlib.reload(B)
+
+
+def test_selftest_wait_timeout_rejects_bad_limits():
+    """The limit is checked on the host before anything touches a device."""
+    lib = B.load()
+    for bad in (0, 1000001):
+        assert lib.wvae_selftest_wait_timeout(bad, NULL) == 1  # WVAE_ERR_INVALID_ARG

@@ -60,7 +60,7 @@ def test_norm_silu_full_size_sampled(shape):
 
 @pytest.mark.parametrize("C,T,H,W", [(512, 4, 87, 91), (64, 4, 176, 330), (1024, 2, 83, 89)])
 def test_norm_silu_many_chunks_ragged(C, T, H, W):
-    """Over 6 x 148 chunks of 32 KB (the 6-stage ring wraps around in every CTA)
+    """Over 3 x 148 chunks of 64 KB (the 3-stage ring wraps around in every CTA)
     and a ragged last chunk; every voxel compared."""
     x, g, b = synth.norm_silu_input(C=C, T=T, H=H, W=W, seed=C + 7)
     y = B.norm_silu(to_cl(x), g.cuda(), b.cuda())

@@ -53,6 +53,7 @@ def load(path: str | None = None):
             "wvae_status_string": (ctypes.c_char_p, [I]),
             "wvae_version": (I, []),
             "wvae_device_error": (I, [ctypes.POINTER(ctypes.c_uint), I]),
+            "wvae_selftest_wait_timeout": (I, [ctypes.c_uint, V]),
             "wvae_norm_silu": (I, [V, V, V, V, I, I, I, I, F, I, V]),
             "wvae_conv_packed_bytes": (S, [I, I, I, I, I, I]),
             "wvae_prepack_conv": (I, [V, I, V, I, I, I, I, I, I, V, S, V]),
@@ -142,6 +143,12 @@ def device_error(reset: bool = True) -> int:
     if st not in (OK, 6):
         raise WvaeError("wvae_device_error", st)
     return code.value
+
+
+def selftest_wait_timeout(limit_us: int = 20000):
+    """Enqueue the bounded-wait self-test (a wait that nothing completes gives
+    up after limit_us and sets bit 0x10 of the device error word)."""
+    _check("wvae_selftest_wait_timeout", load().wvae_selftest_wait_timeout(int(limit_us), _stream()))
 
 
 # ------------------------------------------------------------------ norm-SiLU

@@ -13,9 +13,9 @@
 // full HBM rate), so SiLU costs one SFU operation (tanh form) per element.
 //
 // bf16 (norm_silu_ring_kernel): one persistent CTA per SM.  Warp 0 streams
-// contiguous chunks of whole voxels (about 32 KB: the activation is
-// channels-last, so a chunk is one byte range) into a ring of shared-memory
-// stages with bulk asynchronous copies, keeping ~190 KB per SM in flight
+// contiguous chunks of whole voxels (about 64 KB: the activation is
+// channels-last, so a chunk is one byte range) into a 3-stage ring of
+// shared-memory stages with bulk asynchronous copies, keeping ~190 KB per SM in flight
 // without holding registers; 16 consumer warps take the voxels of each chunk.
 // A group of L lanes owns a voxel (L = 32 for C >= 256) and moves 16-byte
 // vectors, so shared-memory reads and global writes of a voxel are contiguous
@@ -135,8 +135,8 @@ __global__ void __launch_bounds__(kNormThreads, (VEC == 8 && CH <= 4) ? 3 : 2) n
 // ------------------------------------------------------- bf16: TMA-fed ring
 constexpr int kRingWarps = 16;                       // consumer warps
 constexpr int kRingThreads = 32 * (1 + kRingWarps);  // + the copy warp
-constexpr int kRingStages = 6;
-constexpr int kRingChunkBytes = 32768;
+constexpr int kRingStages = 3;
+constexpr int kRingChunkBytes = 65536;
 
 template <int CH>
 __global__ void __launch_bounds__(kRingThreads, 1)
