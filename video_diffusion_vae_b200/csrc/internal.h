@@ -10,11 +10,10 @@
 namespace wvae {
 
 // ----------------------------------------------------------- conv (tcgen05)
-// MMA sub-tile: 128 voxels of one frame, 8 rows x 16 columns (MMA row m =
-// 16 * row + column).  A CTA tile of tile_rows x tile_cols voxels (128 S in
-// all, tile_cols in {16, 32, 64}) is S such sub-tiles of 128 consecutive
-// voxels in row-major order; their S M=128 MMAs share each weight tile.  K
-// block: 64 input channels of one tap.
+// A CTA tile of tile_rows x tile_cols voxels of one frame (16 x 16 or 8 x 32)
+// is S = 2 MMA sub-tiles of kBM = 128 consecutive voxels in row-major order;
+// their M=128 MMAs share each weight tile.  The reduction runs in K groups of
+// kBK = 64 input channels of one (kt, kw) tap column.
 constexpr int kTileH = 8;
 constexpr int kTileW = 16;
 constexpr int kBM = kTileH * kTileW;  // 128
@@ -39,10 +38,12 @@ struct ConvEpilogue {
 };
 
 struct ConvParams {
-  CUtensorMap tmA;   // main input, bf16 [T][H][W][cin_pad], box {64, tile_cols, tile_rows, 1}
-  CUtensorMap tmB;   // main weights, bf16 [cout_pad][taps * cin_pad], box {64, <=256}
+  CUtensorMap tmA;   // main input, bf16 [T][H][W][cin_pad],
+                     // box {64, tile_cols, tile_rows + kh_eff - 1, 1} (the row-tap window)
+  CUtensorMap tmB;   // main weights, bf16 [cout_pad][taps * cin_pad], box {64, BN}
   CUtensorMap tmC;   // cached frames, bf16 [KT-1][H][W][cin_pad], box as tmA (has_cache)
-  CUtensorMap tmA2;  // shortcut input, bf16 [T][H][W][cin2_pad], box as tmA (cin2_pad > 0)
+  CUtensorMap tmA2;  // shortcut input, bf16 [T][H][W][cin2_pad], box {64, tile_cols,
+                     // tile_rows, 1} (cin2_pad > 0)
   CUtensorMap tmB2;  // shortcut weights, bf16 [cout_pad][cin2_pad]
   int T, H, W;
   int cin_pad, cin2_pad;
@@ -53,7 +54,7 @@ struct ConvParams {
                      //    RMS partial sums over distributed shared memory
   int has_cache;
   int BN, n_tiles;
-  int S;             // MMA sub-tiles per CTA tile; S * BN <= 512 TMEM columns
+  int S;             // MMA sub-tiles per CTA tile (2)
   int tile_rows, tile_cols;  // CTA tile, tile_rows * tile_cols = 128 S voxels of one frame
   int kh_eff, kw_eff;  // row / column taps per A window: KH, KW (2, 2 in phase mode; kw_eff
                        // = 1 when the column taps ride in N)
