@@ -36,6 +36,9 @@ METRIC = "res-block conv TFLOP/s (% bf16 peak); norm-SiLU GB/s (% HBM); frames/s
 UNIT = "frames/s"
 T, H, W = 4, 44, 78
 WIDTHS = (512, 512, 256, 128)
+WORKLOAD = ("Wan2.2-shaped decoder trunk: latents [1,48,4,44,78] -> video [1,3,4,704,1248]; "
+            "conv_in, 4 stages of 2 res blocks (widths 512/512/256/128), 3 nearest-2x upsample "
+            "convs, norm_out+SiLU+head conv + 2x2 pixel shuffle")
 ZC = 48
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 512 << 20
@@ -193,9 +196,7 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": T / v * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": "Wan2.2-shaped decoder trunk, latents [1,48,4,44,78] -> video "
-                               "[1,3,4,704,1248], widths 512/512/256/128, 2 res blocks per stage",
-                   "sample": sample},
+        "config": {"workload": WORKLOAD, "sample": sample},
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -488,10 +489,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": max_total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) latents, random weights with the trunk's shapes)",
-            "config": {"workload": "Wan2.2-shaped decoder trunk: latents [1,48,4,44,78] -> video "
-                                   "[1,3,4,704,1248]; conv_in, 4 stages of 2 res blocks (widths "
-                                   "512/512/256/128), 3 nearest-2x upsample convs, norm_out+SiLU+head "
-                                   "conv + 2x2 pixel shuffle",
+            "config": {"workload": WORKLOAD,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "flushed (512 MiB write) before every timed step, outside the step events",
                        "trunk_dense_tflop_per_step": sum(f for _, f in layers) / 1e12},

@@ -203,6 +203,8 @@ __global__ void __launch_bounds__(kRingThreads, 1)
     }
   }
   const float rootC = sqrtf(static_cast<float>(C));
+  const float eps2 = eps * eps;
+  const bool eps2_normal = eps2 >= 1.17549435e-38f;  // FLT_MIN
   uint32_t it = 0;
   for (long ch = blockIdx.x; ch < nchunks; ch += gridDim.x, ++it) {
     const uint32_t st = it % kRingStages, ph = (it / kRingStages) & 1u;
@@ -222,37 +224,36 @@ __global__ void __launch_bounds__(kRingThreads, 1)
       const int vl = vb + grp;
       const bool live = vl < nv;
       const uint4* src = reinterpret_cast<const uint4*>(stage + static_cast<size_t>(vl) * C * 2);
-      uint4 raw[CH];
+      // the lane's channel pairs, unpacked once for both passes
+      float2 xp[CH][4];
       float2 ssa = make_float2(0.0f, 0.0f), ssb = ssa;  // two packed chains
 #pragma unroll
       for (int k = 0; k < CH; ++k) {
         const int vi = sub + k * L;
-        raw[k] = (live && vi < nvec) ? src[vi] : make_uint4(0u, 0u, 0u, 0u);
-        float v[8];
-        unpack<8>(raw[k], v);
-        const float2 p0 = make_float2(v[0], v[1]), p1 = make_float2(v[2], v[3]);
-        const float2 p2 = make_float2(v[4], v[5]), p3 = make_float2(v[6], v[7]);
-        ssa = ffma2(p0, p0, ssa);
-        ssb = ffma2(p1, p1, ssb);
-        ssa = ffma2(p2, p2, ssa);
-        ssb = ffma2(p3, p3, ssb);
+        const uint4 raw = (live && vi < nvec) ? src[vi] : make_uint4(0u, 0u, 0u, 0u);
+        xp[k][0] = make_float2(bf16lo(raw.x), bf16hi(raw.x));
+        xp[k][1] = make_float2(bf16lo(raw.y), bf16hi(raw.y));
+        xp[k][2] = make_float2(bf16lo(raw.z), bf16hi(raw.z));
+        xp[k][3] = make_float2(bf16lo(raw.w), bf16hi(raw.w));
+        ssa = ffma2(xp[k][0], xp[k][0], ssa);
+        ssb = ffma2(xp[k][1], xp[k][1], ssb);
+        ssa = ffma2(xp[k][2], xp[k][2], ssa);
+        ssb = ffma2(xp[k][3], xp[k][3], ssb);
       }
       float ss = (ssa.x + ssa.y) + (ssb.x + ssb.y);
       for (int off = L >> 1; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-      const float r = rootC / fmaxf(sqrtf(ss), eps);
+      // sqrt(C) / max(||x||, eps) = sqrt(C) * rsqrt(max(ss, eps^2)) while eps^2 is normal
+      const float r = eps2_normal ? rootC * rsqrtf(fmaxf(ss, eps2)) : rootC / fmaxf(sqrtf(ss), eps);
       const float2 r2 = make_float2(r, r);
       uint4* dst = reinterpret_cast<uint4*>(y + (v0 + vl) * C);
 #pragma unroll
       for (int k = 0; k < CH; ++k) {
         const int vi = sub + k * L;
         if (!live || vi >= nvec) continue;
-        float v[8];
-        unpack<8>(raw[k], v);
         uint32_t w4[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float2 o = silu_half2(ffma2(make_float2(v[2 * e], v[2 * e + 1]),
-                                            fmul2(r2, g[k][e]), b[k][e]));
+          const float2 o = silu_half2(ffma2(xp[k][e], fmul2(r2, g[k][e]), b[k][e]));
           w4[e] = pack_bf16x2(o.x, o.y);
         }
         dst[vi] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
