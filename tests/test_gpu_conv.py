@@ -17,8 +17,8 @@ def _run(x, w, b, dtype, **kw):
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_conv_tiny_config(dtype):
-    """Config 0's conv: 64 -> 64, x [64, 2, 16, 16]."""
+def test_conv_tiny(dtype):
+    """The tiny workload's conv: 64 -> 64, x [64, 2, 16, 16]."""
     x, w, b = synth.conv_input(cin=64, cout=64, T=2, H=16, W=16, seed=0, bf16=dtype == torch.bfloat16)
     _, y = _run(x, w, b, dtype)
     assert_close(from_cl(y), O.causal_conv3d(x, w, b), dtype, "tiny")
@@ -78,7 +78,7 @@ def test_conv_causality_bitwise():
 
 
 def test_conv_full_size_sampled():
-    """Config 2: 512 -> 512 on [512, 4, 88, 156]; sampled voxels against the oracle."""
+    """512 -> 512 on [512, 4, 88, 156] (full size); sampled voxels against the oracle."""
     x, w, b = synth.conv_input(cin=512, cout=512, T=4, H=88, W=156, seed=0)
     pk = B.prepack_conv(w.cuda().bfloat16(), b.cuda())
     y = B.causal_conv3d(to_cl(x), pk)
@@ -87,7 +87,7 @@ def test_conv_full_size_sampled():
     pts = sample_voxels(4, 88, 156, 48, seed=2)
     got = np.stack([yc[t, h, ww].double().numpy() for (t, h, ww) in pts], 1)
     ref = np.stack([O.causal_conv3d_at(x, w, b, t, h, ww) for (t, h, ww) in pts], 1)
-    assert_close(got, ref, torch.bfloat16, "config 2 sampled")
+    assert_close(got, ref, torch.bfloat16, "512->512 full size sampled")
     assert torch.isfinite(yc).all()
     assert B.device_error() == 0
 

@@ -23,12 +23,12 @@ def resblock_at(x, p, t, h, w):
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_resblock_tiny_config(dtype):
-    """Config 0: x [64, 2, 16, 16], two (norm + SiLU + conv 64->64) stages + identity."""
+def test_resblock_tiny(dtype):
+    """Tiny res block: x [64, 2, 16, 16], two (norm + SiLU + conv 64->64) stages + identity."""
     x, p = synth.tiny_resblock(bf16=dtype == torch.bfloat16)
     blk = B.PackedResBlock(p, dtype)
     y = B.resblock(to_cl(x, dtype), blk)
-    assert_close(from_cl(y), O.resblock(x, p), dtype, "config 0")
+    assert_close(from_cl(y), O.resblock(x, p), dtype, "tiny res block")
 
 
 @pytest.mark.parametrize("cin,cout", [(256, 256), (256, 128), (128, 64), (64, 128), (512, 512)])
@@ -43,7 +43,7 @@ def test_resblock_reduced(cin, cout):
 
 @pytest.mark.parametrize("cout", [256, 128])
 def test_resblock_full_size_sampled(cout):
-    """Config 3 (and its 256 -> 128 shortcut variant) at [256, 4, 176, 312]."""
+    """Res block 256 -> 256 (and the 256 -> 128 shortcut variant) at [256, 4, 176, 312]."""
     x, p = synth.resblock_input(cin=256, cout=cout, T=4, H=176, W=312, seed=0)
     blk = B.PackedResBlock(p)
     y = B.resblock(to_cl(x), blk)
@@ -52,7 +52,7 @@ def test_resblock_full_size_sampled(cout):
     pts = sample_voxels(4, 176, 312, 12, seed=3)
     got = np.stack([yc[t, h, w].double().numpy() for (t, h, w) in pts], 1)
     ref = np.stack([resblock_at(x, p, t, h, w) for (t, h, w) in pts], 1)
-    assert_close(got, ref, torch.bfloat16, f"config 3 cout={cout}")
+    assert_close(got, ref, torch.bfloat16, f"res block 256->{cout}")
     assert torch.isfinite(yc).all()
     assert B.device_error() == 0
 
@@ -129,7 +129,8 @@ def test_trunk_full_width_end_to_end():
 
 
 def test_trunk_full_size_properties():
-    """Config 4 at full size: finite, deterministic, and causal bit for bit."""
+    """The trunk at full size (latents [1, 48, 4, 44, 78]): finite, deterministic, and
+    causal bit for bit."""
     z, params = synth.trunk_input(T=4, H=44, W=78, seed=0)
     tr = B.PackedTrunk(params)
     zd = z[None].cuda().bfloat16().contiguous()
@@ -147,10 +148,10 @@ def test_trunk_full_size_properties():
 
 
 def test_trunk_full_size_vs_standalone_entry_points():
-    """Config 4 at full size, every output element: the fused trunk against the
-    same decoder composed from the standalone entry points (causal conv, res
-    block, upsample conv, norm-SiLU prologue), each checked against the oracle
-    above.  This covers what only full-size layers run (several tiles per CTA,
+    """The trunk at full size (latents [1, 48, 4, 44, 78]), every output element:
+    the fused trunk against the same decoder composed from the standalone entry
+    points (causal conv, res block, upsample conv, norm-SiLU prologue), each
+    checked against the oracle above.  This covers what only full-size layers run (several tiles per CTA,
     the early accumulator release, wave-balanced tile shapes).  The paths round
     differently (fp32 residual stream and fused norms vs bf16 between calls),
     so the bound is the sum of the two paths' bounds against the oracle:
