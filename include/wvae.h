@@ -228,6 +228,32 @@ WVAE_API wvae_status wvae_decode_trunk_timed(const void* const* packed, const fl
                                     size_t ws_bytes, void* const* events, int n_events,
                                     wvae_stream_t stream);
 
+/*
+ * Streaming decode in temporal chunks (the decoder's temporal caching:
+ * TensorRT-LLM issue #19309, "Feature, motivation and proposed scope"; the
+ * FastVideo decoder decodes a few latent frames per pass, README "Use").
+ * Same arguments and work as wvae_decode_trunk on the chunk's T >= 2 latent
+ * frames, plus `cache`: a caller-owned device buffer of
+ * wvae_decode_trunk_cache_bytes(H, W, widths) bytes (16-byte aligned) holding,
+ * for each of the 18 causal 3x3x3 convs (conv_in, the 16 res-block convs, the
+ * head), the last two frames of its input.  With continue_chunk == 0 the
+ * convs see zero front frames (the first chunk) and the cache's content is
+ * ignored; with continue_chunk != 0 they read their front frames from the
+ * cache.  Either way the call leaves the cache holding this chunk's last two
+ * input frames of every causal conv, so decoding latents chunk by chunk
+ * gives the same video as decoding them in one call (the upsample convs are
+ * per frame and need no cache).  Besides the 22 kernels of
+ * wvae_decode_trunk it enqueues 18 device-to-device copies on `stream`.
+ * Returns WVAE_ERR_INVALID_ARG for T < 2 or a NULL cache,
+ * WVAE_ERR_WORKSPACE for a short cache, as wvae_decode_trunk otherwise.
+ */
+WVAE_API size_t wvae_decode_trunk_cache_bytes(int H, int W, const int* widths);
+WVAE_API wvae_status wvae_decode_trunk_chunk(const void* const* packed, const float* const* norms,
+                                    const void* z, void* video, int T, int H, int W,
+                                    const int* widths, wvae_dtype dtype, void* workspace,
+                                    size_t ws_bytes, void* cache, size_t cache_bytes,
+                                    int continue_chunk, wvae_stream_t stream);
+
 /* ------------------------------------------------- res block, no allocation
  * (No counterpart on the pages: this is a convenience of this library.)
  *

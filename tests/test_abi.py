@@ -20,7 +20,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     declared = B.header_symbols()
-    assert len(declared) == 20
+    assert len(declared) == 22
     out = subprocess.check_output(["nm", "-D", "--defined-only", B.LIB_PATH], text=True)
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
     missing = [s for s in declared if s not in exported]
@@ -149,3 +149,24 @@ def test_selftest_wait_timeout_rejects_bad_limits():
     lib = B.load()
     for bad in (0, 1000001):
         assert lib.wvae_selftest_wait_timeout(bad, NULL) == 1  # WVAE_ERR_INVALID_ARG
+
+
+def test_trunk_cache_bytes_and_chunk_validation():
+    """The chunked decode's cache holds two input frames of each of the 18
+    causal convs; T < 2 and a missing cache are refused on the host."""
+    lib = B.load()
+    w = (ctypes.c_int * 4)(512, 512, 256, 128)
+    H, W = 44, 78
+    frames = [H * W * 64] + [(H << s) * (W << s) * c for s, c in enumerate((512, 512, 256, 128))
+                             for _ in range(4)] + [(H << 3) * (W << 3) * 128]
+    want = sum(-(-2 * f * 2 // 256) * 256 for f in frames)
+    assert lib.wvae_decode_trunk_cache_bytes(H, W, w) == want
+    assert lib.wvae_decode_trunk_cache_bytes(0, W, w) == 0
+    P = (ctypes.c_void_p * 21)(*([A] * 21))
+    N = (ctypes.c_void_p * 34)(*([A] * 34))
+    # T = 1 cannot hand two frames on; a NULL cache is refused
+    assert lib.wvae_decode_trunk_chunk(P, N, A, A, 1, H, W, w, B.BF16, A, 1 << 40, A, 1 << 40, 0,
+                                       NULL) == 1
+    assert lib.wvae_decode_trunk_chunk(P, N, A, A, 4, H, W, w, B.BF16, A, 1 << 40, NULL, 0, 0,
+                                       NULL) == 1
+

@@ -196,3 +196,41 @@ def test_trunk_full_size_vs_standalone_entry_points():
     assert rel <= 2e-2, f"rel L2 {rel:.3e}"
     assert mx <= 1e-1, f"max |diff| / std {mx:.3e}"
     assert B.device_error() == 0
+
+
+@pytest.mark.parametrize("chunks", [(2, 4), (3, 3), (2, 2, 2)])
+def test_trunk_chunked_decode_equals_whole(chunks):
+    """Decoding the latents chunk by chunk, each causal conv reading its two
+    front frames from the previous chunk's cache, gives the whole decode's
+    video bit for bit (reduced widths, T = 6)."""
+    T = sum(chunks)
+    z, params = synth.trunk_input(T=T, H=3, W=5, widths=(128, 128, 64, 64), seed=3)
+    tr = B.PackedTrunk(params)
+    zd = z[None].cuda().bfloat16().contiguous()
+    whole = B.decode_trunk(zd, tr)
+    stream = B.TrunkStream(tr, 3, 5)
+    parts, t0 = [], 0
+    for n in chunks:
+        parts.append(stream.decode(zd[:, :, t0:t0 + n].contiguous()))
+        t0 += n
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat(parts, dim=2), whole)
+    assert B.device_error() == 0
+
+
+def test_trunk_chunked_decode_full_size():
+    """Full widths and frames (latents [1, 48, 8, 44, 78]) in two chunks of 4
+    against one decode of all 8 frames, bit for bit; the first chunk's video
+    also equals a fresh 4-frame decode."""
+    z, params = synth.trunk_input(T=8, H=44, W=78, seed=1)
+    tr = B.PackedTrunk(params)
+    zd = z[None].cuda().bfloat16().contiguous()
+    whole = B.decode_trunk(zd, tr)
+    stream = B.TrunkStream(tr, 44, 78)
+    a = stream.decode(zd[:, :, :4].contiguous())
+    b = stream.decode(zd[:, :, 4:].contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(a, whole[:, :, :4])
+    assert torch.equal(b, whole[:, :, 4:])
+    assert torch.equal(a, B.decode_trunk(zd[:, :, :4].contiguous(), tr))
+    assert B.device_error() == 0

@@ -72,6 +72,9 @@ def load(path: str | None = None):
             "wvae_resblock_noalloc": (I, [V, V, I, I, I, I, I, V, V, V, V, V, V, V, V]),
             "wvae_decode_trunk_timed": (I, [ctypes.POINTER(V), ctypes.POINTER(V), V, V, I, I, I,
                                             ctypes.POINTER(I), I, V, S, ctypes.POINTER(V), I, V]),
+            "wvae_decode_trunk_cache_bytes": (S, [I, I, ctypes.POINTER(I)]),
+            "wvae_decode_trunk_chunk": (I, [ctypes.POINTER(V), ctypes.POINTER(V), V, V, I, I, I,
+                                            ctypes.POINTER(I), I, V, S, V, S, I, V]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -311,6 +314,9 @@ class PackedTrunk:
     def workspace_bytes(self, T, H, W):
         return load().wvae_decode_trunk_workspace_bytes(T, H, W, self._widths_arr)
 
+    def cache_bytes(self, H, W):
+        return load().wvae_decode_trunk_cache_bytes(H, W, self._widths_arr)
+
 
 def trunk_launches() -> int:
     return load().wvae_decode_trunk_launches()
@@ -344,3 +350,32 @@ def decode_trunk(z, trunk: PackedTrunk, out=None, workspace=None, events=None):
         trunk._packed_arr, trunk._norm_arr, _ptr(z), _ptr(y), T, H, W, trunk._widths_arr, BF16,
         _ptr(ws), ws.numel(), arr, len(handles), _stream()))
     return y
+
+
+class TrunkStream:
+    """Chunked decode with the causal caches carried between chunks: feeding the
+    latents chunk by chunk gives the video of decoding them at once."""
+
+    def __init__(self, trunk: PackedTrunk, H, W, device="cuda"):
+        self.trunk, self.H, self.W = trunk, H, W
+        self.cache = _workspace(trunk.cache_bytes(H, W), torch.device(device))
+        self.started = False
+
+    def decode(self, z, out=None, workspace=None):
+        """z: the next chunk of latents [1, 48, T, H, W] bf16 (T >= 2) -> its video."""
+        _cuda(z, "z", torch.bfloat16)
+        _, zc, T, H, W = z.shape
+        if zc != 48 or z.shape[0] != 1 or (H, W) != (self.H, self.W):
+            raise ValueError(f"z must be [1, 48, T, {self.H}, {self.W}]")
+        y = torch.empty((1, 3, T, 16 * H, 16 * W), dtype=torch.bfloat16, device=z.device) \
+            if out is None else _cuda(out, "out", torch.bfloat16, (1, 3, T, 16 * H, 16 * W))
+        tr = self.trunk
+        nws = tr.workspace_bytes(T, H, W)
+        ws = _workspace(nws, z.device) if workspace is None else workspace
+        _check("wvae_decode_trunk_chunk", load().wvae_decode_trunk_chunk(
+            tr._packed_arr, tr._norm_arr, _ptr(z), _ptr(y), T, H, W, tr._widths_arr, BF16,
+            _ptr(ws), ws.numel(), _ptr(self.cache), self.cache.numel(), int(self.started),
+            _stream()))
+        self.started = True
+        return y
+

@@ -639,6 +639,47 @@ TrunkBuffers trunk_buffers(int T, int H, int W, const int* C) {
 }
 }  // namespace
 
+namespace {
+// Causal conv inputs whose last two frames a chunk hands to the next one:
+// conv_in, the 16 res-block convs (conv1 and conv2 of 2 blocks x 4 stages),
+// the head.  Offsets into the caller's cache buffer, in that order.
+constexpr int kTrunkCaches = 18;
+
+struct TrunkCaches {
+  size_t off[kTrunkCaches];
+  size_t bytes[kTrunkCaches];
+  size_t total;
+};
+
+TrunkCaches trunk_caches(int H, int W, const int* C) {
+  TrunkCaches c;
+  size_t off = 0;
+  int i = 0;
+  auto take = [&](size_t n) {
+    c.off[i] = off;
+    c.bytes[i] = n;
+    off += round_up_sz(n, 256);
+    ++i;
+  };
+  take(2ull * H * W * kZPad * 2);  // conv_in: padded latents
+  for (int s = 0; s < 4; ++s) {
+    const size_t frame = (static_cast<size_t>(H) << s) * (static_cast<size_t>(W) << s) * C[s] * 2;
+    for (int k = 0; k < 4; ++k) take(2 * frame);  // conv1, conv2 of 2 blocks
+  }
+  take(2ull * (static_cast<size_t>(H) << 3) * (static_cast<size_t>(W) << 3) * C[3] * 2);  // head
+  c.total = off;
+  return c;
+}
+}  // namespace
+
+size_t wvae_decode_trunk_cache_bytes(int H, int W, const int* widths) {
+  if (H < 1 || W < 1) return 0;
+  const int* C = widths ? widths : kDefaultWidths;
+  for (int s = 0; s < 4; ++s)
+    if (C[s] < 64) return 0;
+  return trunk_caches(H, W, C).total;
+}
+
 size_t wvae_decode_trunk_workspace_bytes(int T, int H, int W, const int* widths) {
   if (T < 1 || H < 1 || W < 1) return 0;
   const int* C = widths ? widths : kDefaultWidths;
@@ -650,11 +691,16 @@ size_t wvae_decode_trunk_workspace_bytes(int T, int H, int W, const int* widths)
 namespace {
 constexpr int kTrunkLaunches = 22;
 
+// cache (optional): the causal caches of a chunked decode; continue_chunk:
+// read the front frames from it (else zeros); it is rewritten with this
+// chunk's last two input frames of every causal conv.
 wvae_status decode_trunk_impl(const void* const* packed, const float* const* norms, const void* z,
                               void* video, int T, int H, int W, const int* widths,
                               wvae_dtype dtype, void* workspace, size_t ws_bytes,
-                              void* const* events, int n_events, wvae_stream_t stream) {
+                              void* const* events, int n_events, void* cache, size_t cache_bytes,
+                              int continue_chunk, wvae_stream_t stream) {
   if (!packed || !norms || !z || !video || !workspace) return WVAE_ERR_INVALID_ARG;
+  if (cache != nullptr && T < 2) return WVAE_ERR_INVALID_ARG;  // the cache holds two frames
   if (events != nullptr && n_events < 2 * kTrunkLaunches) return WVAE_ERR_INVALID_ARG;
   if (T < 1 || H < 1 || W < 1) return WVAE_ERR_INVALID_ARG;
   if (dtype != WVAE_BF16) return WVAE_ERR_UNSUPPORTED;
@@ -670,6 +716,11 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
   if (!a16(z) || !a16(video) || !a16(workspace)) return WVAE_ERR_ALIGNMENT;
   const TrunkBuffers B = trunk_buffers(T, H, W, C);
   if (ws_bytes < B.total) return WVAE_ERR_WORKSPACE;
+  const TrunkCaches K = trunk_caches(H, W, C);
+  if (cache != nullptr) {
+    if (!a16(cache)) return WVAE_ERR_ALIGNMENT;
+    if (cache_bytes < K.total) return WVAE_ERR_WORKSPACE;
+  }
   DeviceInfo* d = nullptr;
   wvae_status st = device_info(&d);
   if (st != WVAE_OK) return st;
@@ -685,6 +736,19 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
     mark(1);
     ++launch;
     return r;
+  };
+  // A causal conv of a chunked decode: front frames from cache entry k, then
+  // the last two frames of its input x (T frames of `frame` bytes) become the
+  // next chunk's entry k.
+  int ck = 0;
+  auto causal_conv = [&](TcConv c, size_t frame) {
+    char* entry = cache != nullptr ? static_cast<char*>(cache) + K.off[ck] : nullptr;
+    ++ck;
+    if (entry != nullptr && continue_chunk) c.cache = entry;
+    wvae_status r = conv(c);
+    if (r != WVAE_OK || entry == nullptr) return r;
+    return cuda_status(cudaMemcpyAsync(entry, static_cast<const char*>(c.x) + (T - 2) * frame,
+                                       2 * frame, cudaMemcpyDeviceToDevice, s));
   };
   char* ws = static_cast<char*>(workspace);
   void* zcl = ws + B.zcl;
@@ -723,11 +787,12 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
     c.ep.act = act[0];
     next_norm(&c.ep.gamma, &c.ep.beta);
     c.ep.eps = 1e-12f;
-    st = conv(c);
+    st = causal_conv(c, static_cast<size_t>(H) * W * kZPad * 2);
     if (st != WVAE_OK) return st;
   }
   for (int stg = 0; stg < 4; ++stg) {
     const int Cs = C[stg];
+    const size_t frame = static_cast<size_t>(Hs) * Ws * Cs * 2;  // bf16 activation frame
     for (int blk = 0; blk < 2; ++blk) {
       // conv1: A1 -> A2 (norm2 in the epilogue)
       TcConv c1;
@@ -739,7 +804,7 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
       c1.ep.act = act[1];
       next_norm(&c1.ep.gamma, &c1.ep.beta);
       c1.ep.eps = 1e-12f;
-      st = conv(c1);
+      st = causal_conv(c1, frame);
       if (st != WVAE_OK) return st;
       // conv2: h + conv2(A2) -> h (fp32, in place per voxel) and the next activation
       TcConv c2;
@@ -767,7 +832,7 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
         next_norm(&c2.ep.gamma, &c2.ep.beta);
         c2.ep.eps = 1e-12f;
       }
-      st = conv(c2);
+      st = causal_conv(c2, frame);
       if (st != WVAE_OK) return st;
     }
     if (stg < 3) {
@@ -798,7 +863,7 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
   ch.cout = kHeadOut;
   ch.T = T; ch.H = Hs; ch.W = Ws;
   ch.ep.video = static_cast<__nv_bfloat16*>(video);
-  return conv(ch);
+  return causal_conv(ch, static_cast<size_t>(Hs) * Ws * C[3] * 2);
 }
 }  // namespace
 
@@ -809,7 +874,17 @@ wvae_status wvae_decode_trunk(const void* const* packed, const float* const* nor
                               wvae_dtype dtype, void* workspace, size_t ws_bytes,
                               wvae_stream_t stream) {
   return decode_trunk_impl(packed, norms, z, video, T, H, W, widths, dtype, workspace, ws_bytes,
-                           nullptr, 0, stream);
+                           nullptr, 0, nullptr, 0, 0, stream);
+}
+
+wvae_status wvae_decode_trunk_chunk(const void* const* packed, const float* const* norms,
+                                    const void* z, void* video, int T, int H, int W,
+                                    const int* widths, wvae_dtype dtype, void* workspace,
+                                    size_t ws_bytes, void* cache, size_t cache_bytes,
+                                    int continue_chunk, wvae_stream_t stream) {
+  if (cache == nullptr) return WVAE_ERR_INVALID_ARG;
+  return decode_trunk_impl(packed, norms, z, video, T, H, W, widths, dtype, workspace, ws_bytes,
+                           nullptr, 0, cache, cache_bytes, continue_chunk, stream);
 }
 
 wvae_status wvae_decode_trunk_timed(const void* const* packed, const float* const* norms,
@@ -819,7 +894,7 @@ wvae_status wvae_decode_trunk_timed(const void* const* packed, const float* cons
                                     wvae_stream_t stream) {
   if (events == nullptr) return WVAE_ERR_INVALID_ARG;
   return decode_trunk_impl(packed, norms, z, video, T, H, W, widths, dtype, workspace, ws_bytes,
-                           events, n_events, stream);
+                           events, n_events, nullptr, 0, 0, stream);
 }
 
 // ------------------------------------------------- res block, no allocation
