@@ -485,7 +485,13 @@ __device__ __forceinline__ void result_chunk(const ConvParams& p, const Smem& s,
                                              float (&v)[NC]) {
   tmem_load_chunk<NC>(taddr + c0, v);
 #pragma unroll
-  for (int j = 0; j < NC; ++j) v[j] += s.bias[n0 + c0 + j];
+  for (int q = 0; q < NC / 4; ++q) {  // 128-bit shared loads of the bias
+    const float4 bq = reinterpret_cast<const float4*>(s.bias + n0 + c0)[q];
+    v[4 * q] += bq.x;
+    v[4 * q + 1] += bq.y;
+    v[4 * q + 2] += bq.z;
+    v[4 * q + 3] += bq.w;
+  }
   if (p.ep.residual != nullptr && valid)
     add_residual<NC>(p.ep, vox * p.cout + n0 + c0, v);
 }
@@ -508,8 +514,16 @@ __device__ __forceinline__ void store_act(const ConvParams& p, const Smem& s, in
                                           size_t ovox, float rs, const float (&v)[NC]) {
   // packed pairs: SiLU_half((v rs) gamma/2 + beta/2)
   const float2 r2 = make_float2(rs, rs);
-  const float2* g2 = reinterpret_cast<const float2*>(s.gamma + n0 + c0);
-  const float2* b2 = reinterpret_cast<const float2*>(s.beta + n0 + c0);
+  const float4* g4 = reinterpret_cast<const float4*>(s.gamma + n0 + c0);
+  const float4* b4 = reinterpret_cast<const float4*>(s.beta + n0 + c0);
+  auto g2 = [&](int i) {  // channel pair i as two lanes of a 128-bit load
+    const float4 g = g4[i >> 1];
+    return (i & 1) ? make_float2(g.z, g.w) : make_float2(g.x, g.y);
+  };
+  auto b2 = [&](int i) {
+    const float4 b = b4[i >> 1];
+    return (i & 1) ? make_float2(b.z, b.w) : make_float2(b.x, b.y);
+  };
   __nv_bfloat16* dst = p.ep.act + ovox * p.cout + n0 + c0;
   if (p.ep.vec32) {
 #pragma unroll
@@ -519,7 +533,7 @@ __device__ __forceinline__ void store_act(const ConvParams& p, const Smem& s, in
       for (int e = 0; e < 8; ++e) {
         const int j = 16 * q + 2 * e;
         const float2 o =
-            silu_half2(ffma2(fmul2(make_float2(v[j], v[j + 1]), r2), g2[j / 2], b2[j / 2]));
+            silu_half2(ffma2(fmul2(make_float2(v[j], v[j + 1]), r2), g2(j / 2), b2(j / 2)));
         w[e] = pack_bf16x2(o.x, o.y);
       }
       st_global_v8(dst + 16 * q, w);
@@ -534,7 +548,7 @@ __device__ __forceinline__ void store_act(const ConvParams& p, const Smem& s, in
     for (int e = 0; e < 4; ++e) {
       const int j = 8 * q + 2 * e;
       const float2 o =
-          silu_half2(ffma2(fmul2(make_float2(v[j], v[j + 1]), r2), g2[j / 2], b2[j / 2]));
+          silu_half2(ffma2(fmul2(make_float2(v[j], v[j + 1]), r2), g2(j / 2), b2(j / 2)));
       w[e] = pack_bf16x2(o.x, o.y);
     }
     d[q] = make_uint4(w[0], w[1], w[2], w[3]);
