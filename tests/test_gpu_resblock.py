@@ -234,3 +234,18 @@ def test_trunk_chunked_decode_full_size():
     assert torch.equal(b, whole[:, :, 4:])
     assert torch.equal(a, B.decode_trunk(zd[:, :, :4].contiguous(), tr))
     assert B.device_error() == 0
+
+
+def test_trunk_cuda_graph_replay():
+    """The trunk captured once as a CUDA graph replays to the direct decode's
+    video, also after new latents are copied into its input buffer."""
+    z, params = synth.trunk_input(T=3, H=3, W=5, widths=(128, 128, 64, 64), seed=4)
+    z2, _ = synth.trunk_input(T=3, H=3, W=5, widths=(128, 128, 64, 64), seed=5)
+    tr = B.PackedTrunk(params)
+    zd = z[None].cuda().bfloat16().contiguous()
+    zd2 = z2[None].cuda().bfloat16().contiguous()
+    g = B.TrunkGraph(tr, zd.clone())
+    assert torch.equal(g.replay().clone(), B.decode_trunk(zd, tr))
+    g.z.copy_(zd2)
+    assert torch.equal(g.replay().clone(), B.decode_trunk(zd2, tr))
+    assert B.device_error() == 0

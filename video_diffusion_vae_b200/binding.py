@@ -379,3 +379,26 @@ class TrunkStream:
         self.started = True
         return y
 
+
+
+class TrunkGraph:
+    """One trunk decode captured as a CUDA graph on fixed buffers: replay()
+    re-runs its 22 launches with a single host call (copy the next latents into
+    `.z` first).  The library's host work (tensor-map encoding, launch
+    configuration) happens once, at capture."""
+
+    def __init__(self, trunk: PackedTrunk, z):
+        _cuda(z, "z", torch.bfloat16)
+        self.z = z
+        _, _, T, H, W = z.shape
+        self.out = torch.empty((1, 3, T, 16 * H, 16 * W), dtype=torch.bfloat16, device=z.device)
+        self.ws = _workspace(trunk.workspace_bytes(T, H, W), z.device)
+        decode_trunk(self.z, trunk, out=self.out, workspace=self.ws)  # device set-up, kernel attributes
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            decode_trunk(self.z, trunk, out=self.out, workspace=self.ws)
+
+    def replay(self):
+        self.graph.replay()
+        return self.out
