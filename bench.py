@@ -110,59 +110,127 @@ def conv_traffic():
 
 # ------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples (200 ms) of SM clock and throttle reasons during a region."""
+    """SM clock and clock-event (throttle) reasons sampled while a region runs.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NVML is polled every `period_s` from a thread (read-only queries), so even a
+    timed region of a fraction of a second gets a dozen samples; without NVML,
+    nvidia-smi at 100 ms.  Either way the first sample is taken before the
+    region starts."""
 
-    def __init__(self, device_index):
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4),
+               ("hw_power_brake_slowdown", 0x80))
+    SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index, period_s=0.02, nvml=None):
         self.idx = device_index
-        self.proc = None
-        self.path = None
+        self.period = period_s
+        self.nvml = nvml          # a module with pynvml's interface (tests pass a fake)
+        self.rows = []            # (sm_mhz, max_mhz, reason names)
+        self.source = None
+        self._stop = None
+        self._thread = None
+        self._proc = None
+        self._path = None
 
-    def __enter__(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
+    # ---- NVML
+    def _handle(self, nv):
+        try:
+            import torch
+            pr = torch.cuda.get_device_properties(self.idx)
+            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.idx)
+
+    def _sample(self, nv, h):
+        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+        self.rows.append((float(sm), float(mx), [n for n, b in self.REASONS if bits & b]))
+
+    def _poll(self, nv, h):
+        while not self._stop.wait(self.period):
+            try:
+                self._sample(nv, h)
+            except Exception:
+                return
+
+    def _start_nvml(self):
+        import threading
+        nv = self.nvml
+        if nv is None:
+            import pynvml as nv
+        nv.nvmlInit()
+        h = self._handle(nv)
+        self._sample(nv, h)  # first sample before the region
+        self._stop = threading.Event()
+        self._thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+        self._thread.start()
+        self.source = "nvml"
+
+    # ---- nvidia-smi
+    def _start_smi(self):
+        fd, self._path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.SMI_FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                stdout=open(self._path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
-            self.proc = None
+            os.unlink(self._path)
+            raise
+        t0 = time.time()
+        while time.time() - t0 < 3.0 and os.path.getsize(self._path) == 0:
+            time.sleep(0.02)
+        self.source = "nvidia-smi"
+
+    def _read_smi(self):
+        names = [n for n, _ in self.REASONS[:4]]
+        try:
+            for line in open(self._path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9 or not f[1].replace(".", "").isdigit():
+                    continue
+                mx = float(f[2]) if f[2].replace(".", "").isdigit() else float("nan")
+                self.rows.append((float(f[1]), mx,
+                                  [names[i] for i in range(4) if f[5 + i].lower() == "active"]))
+        finally:
+            os.unlink(self._path)
+
+    def __enter__(self):
+        try:
+            self._start_nvml()
+        except Exception:
+            try:
+                self._start_smi()
+            except Exception:
+                self._proc = None
         return self
 
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+        if self._proc is not None:
+            self._proc.terminate()
             try:
-                self.proc.wait(timeout=5)
+                self._proc.wait(timeout=5)
             except Exception:
-                self.proc.kill()
+                self._proc.kill()
+            self._read_smi()
 
     def summary(self):
-        rows = []
-        try:
-            for line in open(self.path):
-                f = [x.strip() for x in line.split(",")]
-                if len(f) >= 9:
-                    rows.append(f)
-        except Exception:
-            pass
-        finally:
-            try:
-                os.unlink(self.path)
-            except Exception:
-                pass
-        if not rows:
+        if not self.rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+        sm = [r[0] for r in self.rows]
+        mx = [r[1] for r in self.rows if r[1] == r[1]]
+        reasons = sorted({n for r in self.rows for n in r[2]})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows), "source": self.source}
 
 
 # ----------------------------------------------------------- CPU baseline
