@@ -273,6 +273,14 @@ def run_reference(args, rank, world):
 
 
 # -------------------------------------------------------------- components
+def flush_l2(buf):
+    """Evict L2 before a timed step: write a buffer larger than L2, then read it
+    back, so that L2 holds none of the step's inputs and no dirty line of the
+    flush (whose write-back would otherwise fall inside the timed step)."""
+    buf.zero_()
+    buf.sum()
+
+
 def time_events(fn, reps, warm, flush):
     import torch
     for _ in range(warm):
@@ -280,7 +288,7 @@ def time_events(fn, reps, warm, flush):
     torch.cuda.synchronize()
     ts = []
     for _ in range(reps):
-        flush.zero_()
+        flush_l2(flush)
         s = torch.cuda.Event(enable_timing=True)
         e = torch.cuda.Event(enable_timing=True)
         s.record()
@@ -459,7 +467,7 @@ def main():
     with ClockSampler(torch.cuda.current_device()) as clk:
         t0 = time.perf_counter()
         for i in range(args.steps):
-            flush.zero_()
+            flush_l2(flush)
             step_ev[i][0].record()
             step()
             step_ev[i][1].record()
@@ -477,7 +485,7 @@ def main():
     # them between its launches) for the per-launch durations; not in `value`
     torch.cuda.synchronize()
     for i in range(args.steps):
-        flush.zero_()
+        flush_l2(flush)
         B.decode_trunk(zd, tr, out=video, workspace=ws, events=ev[i])
     torch.cuda.synchronize()
 
@@ -559,7 +567,7 @@ def main():
             "data": "synthetic (seeded N(0,1) latents, random weights with the trunk's shapes)",
             "config": {"workload": WORKLOAD,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "flushed (512 MiB write) before every timed step, outside the step events",
+                       "l2": "flushed before every timed step, outside the step events (512 MiB written, then read back: no dirty line of the flush left)",
                        "trunk_dense_tflop_per_step": sum(f for _, f in layers) / 1e12},
             "tflops": sum(f for _, f in layers) * args.steps / (total_ms * 1e-3) / 1e12,
             "roofline": {"bound": "tensor", "kernel": "conv_tc_kernel (all 21 conv launches of a step)",
