@@ -135,6 +135,19 @@ def _workspace(nbytes, device):
     return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
 
 
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
+def _ws(workspace, nbytes, device):
+    """The caller's workspace (a contiguous CUDA tensor of any dtype: its size in
+    bytes goes to the library, which rejects one that is too small), else a new
+    one of nbytes on device."""
+    if workspace is None:
+        return _workspace(nbytes, device)
+    return _cuda(workspace, "workspace")
+
+
 def version() -> int:
     return load().wvae_version()
 
@@ -260,11 +273,11 @@ def resblock(x, blk: PackedResBlock, out=None, workspace=None):
         _cuda(out, "out", x.dtype, (T, H, W, cout))
     lib = load()
     nws = lib.wvae_resblock_workspace_bytes(T, H, W, cin, cout, dt)
-    ws = _workspace(nws, x.device) if workspace is None else workspace
+    ws = _ws(workspace, nws, x.device)
     _check("wvae_resblock", lib.wvae_resblock(
         _ptr(x), _ptr(y), T, H, W, cin, cout, _ptr(blk.gamma1), _ptr(blk.beta1), blk.w1.ptr(),
         _ptr(blk.gamma2), _ptr(blk.beta2), blk.w2.ptr(), None if blk.ws is None else blk.ws.ptr(),
-        dt, _ptr(ws), ws.numel(), _stream()))
+        dt, _ptr(ws), _nbytes(ws), _stream()))
     return y
 
 
@@ -333,12 +346,11 @@ def decode_trunk(z, trunk: PackedTrunk, out=None, workspace=None, events=None):
         raise ValueError("z must be [1, 48, T, H, W]")
     y = torch.empty((1, 3, T, 16 * H, 16 * W), dtype=torch.bfloat16, device=z.device) if out is None \
         else _cuda(out, "out", torch.bfloat16, (1, 3, T, 16 * H, 16 * W))
-    nws = trunk.workspace_bytes(T, H, W)
-    ws = _workspace(nws, z.device) if workspace is None else workspace
+    ws = _ws(workspace, trunk.workspace_bytes(T, H, W), z.device)
     if events is None:
         _check("wvae_decode_trunk", load().wvae_decode_trunk(
             trunk._packed_arr, trunk._norm_arr, _ptr(z), _ptr(y), T, H, W, trunk._widths_arr, BF16,
-            _ptr(ws), ws.numel(), _stream()))
+            _ptr(ws), _nbytes(ws), _stream()))
         return y
     handles = []
     for ev in events:
@@ -348,7 +360,7 @@ def decode_trunk(z, trunk: PackedTrunk, out=None, workspace=None, events=None):
     arr = (ctypes.c_void_p * len(handles))(*handles)
     _check("wvae_decode_trunk_timed", load().wvae_decode_trunk_timed(
         trunk._packed_arr, trunk._norm_arr, _ptr(z), _ptr(y), T, H, W, trunk._widths_arr, BF16,
-        _ptr(ws), ws.numel(), arr, len(handles), _stream()))
+        _ptr(ws), _nbytes(ws), arr, len(handles), _stream()))
     return y
 
 
@@ -370,11 +382,10 @@ class TrunkStream:
         y = torch.empty((1, 3, T, 16 * H, 16 * W), dtype=torch.bfloat16, device=z.device) \
             if out is None else _cuda(out, "out", torch.bfloat16, (1, 3, T, 16 * H, 16 * W))
         tr = self.trunk
-        nws = tr.workspace_bytes(T, H, W)
-        ws = _workspace(nws, z.device) if workspace is None else workspace
+        ws = _ws(workspace, tr.workspace_bytes(T, H, W), z.device)
         _check("wvae_decode_trunk_chunk", load().wvae_decode_trunk_chunk(
             tr._packed_arr, tr._norm_arr, _ptr(z), _ptr(y), T, H, W, tr._widths_arr, BF16,
-            _ptr(ws), ws.numel(), _ptr(self.cache), self.cache.numel(), int(self.started),
+            _ptr(ws), _nbytes(ws), _ptr(self.cache), _nbytes(self.cache), int(self.started),
             _stream()))
         self.started = True
         return y
