@@ -126,4 +126,72 @@ def test_pins_catch_shortcut_on_normalised_input():
 
 
 def test_real_oracle_passes_everything():
-    assert not _fails(O, extra=[lambda o: P.check_resblock_library(o, synth)])
+    assert not _fails(O, extra=[lambda o: P.check_resblock_library(o, synth),
+                                lambda o: P.check_trunk_library(o, synth)])
+
+
+# ------------------------------------------------- the causal cache
+def conv_cache_reversed(x, wt, bias=None, cache=None, threads=None):
+    # the cached frames taken newest first
+    c = None if cache is None else np.ascontiguousarray(np.asarray(cache)[:, ::-1])
+    return O.causal_conv3d(x, wt, bias, c, threads)
+
+
+def conv_cache_ignored(x, wt, bias=None, cache=None, threads=None):
+    return O.causal_conv3d(x, wt, bias, None, threads)
+
+
+@pytest.mark.parametrize("mutant", [conv_cache_reversed, conv_cache_ignored])
+def test_pins_catch_cache_mutant(mutant):
+    assert _fails(_ns(causal_conv3d=mutant))
+
+
+# ------------------------------------------------- the trunk's composition
+def trunk_built(z, params, conv_before_upsample=False, head_norm=True,
+                shuffle=O.pixel_shuffle2x2, drop_last_block=False):
+    """The trunk from the oracle's layers, with one composition mistake planted
+    on request (all False / default: the trunk as the oracle defines it)."""
+    h = O.causal_conv3d(z, *params["conv_in"])
+    stages = params["stages"]
+    for s, st in enumerate(stages):
+        blocks = st["blocks"][:-1] if drop_last_block and s == len(stages) - 1 else st["blocks"]
+        for bp in blocks:
+            h = O.resblock(h, bp)
+        if st["up"] is not None:
+            w, b = st["up"]
+            h = O.upsample_nearest2x(O.causal_conv3d(h, w, b)) if conv_before_upsample \
+                else O.causal_conv3d(O.upsample_nearest2x(h), w, b)
+    hp = params["head"]
+    if head_norm:
+        a = O.norm_silu(h, hp["gamma"], hp["beta"])
+    else:
+        s_ = np.asarray(h) * np.asarray(hp["gamma"]).reshape(-1, 1, 1, 1) + \
+            np.asarray(hp["beta"]).reshape(-1, 1, 1, 1)
+        a = s_ / (1 + np.exp(-s_))
+    return shuffle(O.causal_conv3d(a, hp["w"], hp["b"]))
+
+
+TRUNK_MUTANTS = {
+    "conv_before_upsample": dict(conv_before_upsample=True),
+    "head_without_norm": dict(head_norm=False),
+    "head_shuffle_swapped": dict(shuffle=shuffle_swapped),
+    "last_block_dropped": dict(drop_last_block=True),
+}
+
+
+def _trunk_fails(**mistake):
+    ns = types.SimpleNamespace(trunk=lambda z, params, threads=None: trunk_built(z, params, **mistake))
+    try:
+        P.check_trunk_library(ns, synth)
+    except AssertionError:
+        return True
+    return False
+
+
+def test_trunk_rebuild_without_mistake_passes():
+    assert not _trunk_fails()
+
+
+@pytest.mark.parametrize("name", sorted(TRUNK_MUTANTS))
+def test_pins_catch_trunk_mutant(name):
+    assert _trunk_fails(**TRUNK_MUTANTS[name]), f"the trunk pin passed planted mistake {name}"
