@@ -1,0 +1,120 @@
+"""The row-slab split (video_diffusion_vae_b200/shard.py) on the CPU: gloo
+ranks decode their rows of one video through the oracle's layers, exchanging
+one halo row before every 3x3 conv, and each rank's video rows equal the same
+rows of the whole oracle decode, bit for bit."""
+import datetime
+import os
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from video_diffusion_vae_b200 import shard
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_partition():
+    for H, world in [(44, 1), (44, 2), (44, 3), (44, 8), (5, 3), (7, 7)]:
+        parts = shard.partition(H, world)
+        assert parts[0][0] == 0 and parts[-1][1] == H
+        assert all(a[1] == b[0] for a, b in zip(parts, parts[1:]))
+        sizes = [r1 - r0 for r0, r1 in parts]
+        assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
+    assert shard.rows_at((11, 22), 16) == (176, 352)
+    with pytest.raises(ValueError):
+        shard.partition(3, 4)
+
+
+# ---------------------------------------------------------------- gloo ranks
+def _conv_rows(O, a, w, b, rank, world):
+    """A 3x3 conv of this rank's rows: the input gets its halo, the conv runs
+    over rows + 2 and the own rows are kept."""
+    ext = shard.with_halo(torch.from_numpy(np.ascontiguousarray(a)), 2)
+    shard.exchange_halo(ext, rank, world, 2)
+    return O.causal_conv3d(ext.numpy(), w, b)[:, :, 1:-1]
+
+
+def _upconv_rows(O, x, w, b, rank, world):
+    ext = shard.with_halo(torch.from_numpy(np.ascontiguousarray(x)), 2)
+    shard.exchange_halo(ext, rank, world, 2)
+    return O.causal_conv3d(O.upsample_nearest2x(ext.numpy()), w, b)[:, :, 2:-2]
+
+
+def _trunk_rows(O, z, params, rank, world, norm_after_exchange=False):
+    def act(h, g, b):
+        return O.norm_silu(h, g, b)
+
+    def conv_act(h, g, b, w, bias):
+        if norm_after_exchange:
+            # a planted mistake: exchange the raw tensor and normalise the halo
+            # too, so the frame's zero padding turns into SiLU(beta)
+            ext = shard.with_halo(torch.from_numpy(np.ascontiguousarray(h)), 2)
+            shard.exchange_halo(ext, rank, world, 2)
+            return O.causal_conv3d(act(ext.numpy(), g, b), w, bias)[:, :, 1:-1]
+        return _conv_rows(O, act(h, g, b), w, bias, rank, world)
+
+    h = _conv_rows(O, z, *params["conv_in"], rank, world)
+    for st in params["stages"]:
+        for p in st["blocks"]:
+            h1 = conv_act(h, p["gamma1"], p["beta1"], p["w1"], p["b1"])
+            h2 = conv_act(h1, p["gamma2"], p["beta2"], p["w2"], p["b2"])
+            skip = O.causal_conv3d(h, p["ws"], p["bs"]) if p.get("ws") is not None else h
+            h = h2 + skip
+        if st["up"] is not None:
+            h = _upconv_rows(O, h, *st["up"], rank, world)
+    hp = params["head"]
+    return O.pixel_shuffle2x2(conv_act(h, hp["gamma"], hp["beta"], hp["w"], hp["b"]))
+
+
+def _rank(rank, world, port, H, q, norm_after_exchange):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    from oracle import oracle as O
+    from video_diffusion_vae_b200 import synth
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        z, params = synth.trunk_input(T=2, H=H, W=4, widths=(16, 16, 8, 8), zc=6, seed=7)
+        r0, r1 = shard.partition(H, world)[rank]
+        zs = np.asarray(z.double().numpy())[:, :, r0:r1]
+        mine = _trunk_rows(O, zs, params, rank, world, norm_after_exchange)
+        whole = O.trunk(z, params)
+        v0, v1 = shard.rows_at((r0, r1), 16)
+        q.put((rank, mine.shape == whole[:, :, v0:v1].shape and np.array_equal(mine, whole[:, :, v0:v1])))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _run(world, port, H, norm_after_exchange=False):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    ps = [ctx.Process(target=_rank, args=(r, world, port, H, q, norm_after_exchange))
+          for r in range(world)]
+    for p in ps:
+        p.start()
+    for p in ps:
+        p.join(240)
+    for p in ps:          # a rank stuck past the limit is ended, then reported
+        if p.is_alive():
+            p.terminate()
+            p.join(10)
+    assert all(p.exitcode == 0 for p in ps), [p.exitcode for p in ps]
+    return dict(q.get(timeout=10) for _ in range(world))
+
+
+@pytest.mark.parametrize("world,port", [(2, 29631), (3, 29632)])
+def test_row_split_trunk_equals_whole(world, port):
+    got = _run(world, port, H=5)
+    assert all(got.values()), got
+
+
+def test_row_split_needs_the_activated_halo():
+    """Exchanging the raw tensor and normalising the halo rows as well gives
+    the wrong border (SiLU(beta) where the frame pads with zeros)."""
+    got = _run(2, 29633, H=4, norm_after_exchange=True)
+    assert not all(got.values())

@@ -1,0 +1,86 @@
+"""Row-slab split of one decode over ranks: the host side of a spatial split.
+
+The FastVideo Wan2.2 VAE decoder spreads one decode over several GPUs of a
+node - every rank calls it with the same latents, rank 0 receives the video
+(README, "Use"), 3.57x faster at 4 GPUs ("Performance and memory") - without
+saying how it splits the work.  This module holds the host side of a split
+over frame rows:
+
+* partition(): the latent rows each rank owns.  At stage s of the trunk a rank
+  owns the rows [2^s r0, 2^s r1) of that stage's resolution and, in the video,
+  the rows [16 r0, 16 r1).
+* exchange_halo(): the one-row halo every 3x3 conv needs (the causal 3x3x3
+  convs, the upsample convs, the head).  A rank keeps each conv input with
+  one extra row above and below its own rows; before the conv the extra rows
+  are filled with the neighbours' edge rows, or with zeros at the frame's
+  top and bottom.  The exchanged tensor is the conv's INPUT after norm and
+  SiLU, since the frame's zero padding applies after the activation.
+  Everything else on the path (norm, SiLU, residual, shortcut, pixel
+  shuffle) is per voxel and needs no exchange.
+
+With the extra rows in place a conv computed over rows + 2 rows gives its own
+rows exactly (the two outer rows are discarded, or overwritten by the next
+exchange), so the convs themselves need no change.  Works on CPU tensors
+(gloo) and CUDA tensors (NCCL) alike.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+
+def partition(H: int, world: int) -> list[tuple[int, int]]:
+    """Contiguous row ranges [r0, r1) of H rows over `world` ranks, sizes
+    differing by at most one (the first H % world ranks take the extra row)."""
+    if world < 1 or H < world:
+        raise ValueError(f"cannot split {H} rows over {world} ranks")
+    base, extra = divmod(H, world)
+    out, r0 = [], 0
+    for r in range(world):
+        r1 = r0 + base + (1 if r < extra else 0)
+        out.append((r0, r1))
+        r0 = r1
+    return out
+
+
+def rows_at(part: tuple[int, int], scale: int) -> tuple[int, int]:
+    """A rank's rows at a resolution `scale` times the latents'."""
+    return part[0] * scale, part[1] * scale
+
+
+def with_halo(x: torch.Tensor, row_dim: int) -> torch.Tensor:
+    """A copy of x with one (zero) row added above and below along row_dim."""
+    shape = list(x.shape)
+    shape[row_dim] += 2
+    out = x.new_zeros(shape)
+    out.narrow(row_dim, 1, x.shape[row_dim]).copy_(x)
+    return out
+
+
+def exchange_halo(x_ext: torch.Tensor, rank: int, world: int, row_dim: int, group=None) -> None:
+    """Fill the halo rows of x_ext in place.
+
+    x_ext holds, along row_dim, one halo row, the rank's own rows, one halo row.
+    Row 0 receives the last own row of rank - 1 (zeros on rank 0); the last row
+    receives the first own row of rank + 1 (zeros on the last rank).  Every
+    rank of the group must call it (ranks with one neighbour exchange with it
+    alone)."""
+    n = x_ext.shape[row_dim]
+    if n < 3:
+        raise ValueError("x_ext needs at least one own row between the two halo rows")
+    first = x_ext.narrow(row_dim, 1, 1).contiguous()
+    last = x_ext.narrow(row_dim, n - 2, 1).contiguous()
+    top = torch.zeros_like(first)
+    bottom = torch.zeros_like(first)
+    ops = []
+    if rank > 0:
+        ops.append(dist.P2POp(dist.isend, first, rank - 1, group))
+        ops.append(dist.P2POp(dist.irecv, top, rank - 1, group))
+    if rank < world - 1:
+        ops.append(dist.P2POp(dist.isend, last, rank + 1, group))
+        ops.append(dist.P2POp(dist.irecv, bottom, rank + 1, group))
+    if ops:
+        for req in dist.batch_isend_irecv(ops):
+            req.wait()
+    x_ext.narrow(row_dim, 0, 1).copy_(top)
+    x_ext.narrow(row_dim, n - 1, 1).copy_(bottom)
