@@ -29,6 +29,21 @@ def test_partition():
         shard.partition(3, 4)
 
 
+def test_single_rank_halo_is_the_frame_padding():
+    """One rank: both halo rows are the frame's zero padding (no process group
+    needed); channels-last layout, rows on dim 1."""
+    x = torch.randn(2, 3, 5, 8)                       # [T, rows, W, C]
+    ext = shard.with_halo(x, 1)
+    ext[:, 0] = 7.0
+    ext[:, -1] = 7.0
+    shard.exchange_halo(ext, 0, 1, 1)
+    assert ext.shape == (2, 5, 5, 8)
+    assert torch.equal(ext[:, 1:-1], x)
+    assert not ext[:, 0].any() and not ext[:, -1].any()
+    with pytest.raises(ValueError):
+        shard.exchange_halo(torch.zeros(2, 2, 5, 8), 0, 1, 1)
+
+
 # ---------------------------------------------------------------- gloo ranks
 def _conv_rows(O, a, w, b, rank, world):
     """A 3x3 conv of this rank's rows: the input gets its halo, the conv runs
