@@ -1,7 +1,8 @@
 """The row-slab split (video_diffusion_vae_b200/shard.py) on the CPU: gloo
 ranks decode their rows of one video through the oracle's layers, exchanging
-one halo row before every 3x3 conv, and each rank's video rows equal the same
-rows of the whole oracle decode, bit for bit."""
+one halo row before every 3x3 conv; each rank's video rows equal the same
+rows of the whole oracle decode, bit for bit, and rank 0 gathers the whole
+video."""
 import datetime
 import os
 import sys
@@ -99,7 +100,14 @@ def _rank(rank, world, port, H, q, norm_after_exchange):
         mine = _trunk_rows(O, zs, params, rank, world, norm_after_exchange)
         whole = O.trunk(z, params)
         v0, v1 = shard.rows_at((r0, r1), 16)
-        q.put((rank, mine.shape == whole[:, :, v0:v1].shape and np.array_equal(mine, whole[:, :, v0:v1])))
+        ok = mine.shape == whole[:, :, v0:v1].shape and np.array_equal(mine, whole[:, :, v0:v1])
+        video = shard.gather_rows(torch.from_numpy(np.ascontiguousarray(mine)),
+                                  shard.partition(H, world), 16, rank, world, 2)
+        if rank == 0:
+            ok = ok and np.array_equal(video.numpy(), whole)
+        else:
+            ok = ok and video is None
+        q.put((rank, ok))
     finally:
         dist.barrier()
         dist.destroy_process_group()

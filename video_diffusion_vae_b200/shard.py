@@ -9,6 +9,8 @@ over frame rows:
 * partition(): the latent rows each rank owns.  At stage s of the trunk a rank
   owns the rows [2^s r0, 2^s r1) of that stage's resolution and, in the video,
   the rows [16 r0, 16 r1).
+* gather_rows(): rank 0 assembles the whole output from the ranks' rows
+  (the pages' decoder returns the video on rank 0).
 * exchange_halo(): the one-row halo every 3x3 conv needs (the causal 3x3x3
   convs, the upsample convs, the head).  A rank keeps each conv input with
   one extra row above and below its own rows; before the conv the extra rows
@@ -84,3 +86,26 @@ def exchange_halo(x_ext: torch.Tensor, rank: int, world: int, row_dim: int, grou
             req.wait()
     x_ext.narrow(row_dim, 0, 1).copy_(top)
     x_ext.narrow(row_dim, n - 1, 1).copy_(bottom)
+
+
+def gather_rows(mine: torch.Tensor, parts: list[tuple[int, int]], scale: int, rank: int,
+                world: int, row_dim: int, group=None):
+    """Rank 0 receives every rank's rows (`mine`: this rank's rows at `scale`
+    times the latent resolution, along row_dim) and returns the whole tensor;
+    the other ranks send theirs and return None.  Every rank of the group must
+    call it."""
+    r0, r1 = rows_at(parts[rank], scale)
+    if mine.shape[row_dim] != r1 - r0:
+        raise ValueError(f"rank {rank} holds {mine.shape[row_dim]} rows, its part has {r1 - r0}")
+    if rank != 0:
+        dist.send(mine.contiguous(), 0, group)
+        return None
+    pieces = [mine.contiguous()]
+    for src in range(1, world):
+        a, b = rows_at(parts[src], scale)
+        shape = list(mine.shape)
+        shape[row_dim] = b - a
+        buf = mine.new_empty(shape)
+        dist.recv(buf, src, group)
+        pieces.append(buf)
+    return torch.cat(pieces, dim=row_dim)
