@@ -18,7 +18,9 @@ is defined:
   accumulation; temporal caching named in the TensorRT-LLM issue's scope);
 * residual block h = x + conv2(A2(conv1(A1(x)))), with a 1x1x1 shortcut conv
   on the raw input when the channel count changes;
-* nearest 2x upsample followed by a per-frame 3x3 conv between stages;
+* nearest 2x upsample followed by a per-frame 3x3 conv between stages, and
+  (optionally) a temporal 2x upsample after the first two of them, giving
+  4T - 3 video frames;
 * the trunk: conv_in, three (2 res blocks, upsample conv) stages, 2 res blocks,
   norm_out + SiLU + causal conv to 12 channels and a 2x2 pixel shuffle into
   the 3-channel video (FastVideo README intro: 48 latent channels, 16x16
@@ -162,6 +164,24 @@ def resblock(x, p, threads: int | None = None):
     return h2 + skip
 
 
+def temporal_upsample2x(x, first_chunk: bool = True):
+    """Temporal 2x upsample of the causal decoder, shape only (nearest in time).
+
+    The pages fix only the frame counts: latents [1, 48, T, ...] decode to
+    4T - 3 video frames (FastVideo Wan2.2 VAE decoder README, opening section:
+    4x temporal compression, video [1, 3, 4T - 3, 704, 1248]).  Read as two
+    2x steps, each keeping the decode's first frame once (the causal first
+    frame has no predecessor to pair with) and turning every later frame into
+    two consecutive copies: T frames -> 2T - 1, and twice -> 4T - 3.  A chunk
+    of a streaming decode that is not the first (first_chunk=False) holds no
+    first frame, so all of its T frames double: T -> 2T.  x: [C, T, H, W]."""
+    x = _f64(x)
+    src = []
+    for t in range(x.shape[1]):
+        src += [t] if (t == 0 and first_chunk) else [t, t]
+    return np.ascontiguousarray(x[:, src])
+
+
 def upsample_conv(x, wt, bias, threads: int | None = None):
     """Nearest 2x upsample, then a per-frame 3x3 conv (KT = 1) with zero border."""
     return causal_conv3d(upsample_nearest2x(x), wt, bias, threads=threads)
@@ -173,11 +193,18 @@ def head(h, gamma, beta, wt, bias, threads: int | None = None):
     return pixel_shuffle2x2(causal_conv3d(a, wt, bias, threads=threads))
 
 
-def trunk(z, params, threads: int | None = None, trace: dict | None = None):
+def trunk(z, params, threads: int | None = None, trace: dict | None = None,
+          temporal: bool = False, first_chunk: bool = True):
     """Decoder trunk.  params: 'conv_in' -> (w, b); 'stages' -> list of dicts
     {'blocks': [resblock params...], 'up': (w, b) or None}; 'head' -> dict
-    gamma, beta, w, b.  Returns the video [3, T, 2H', 2W'].  If ``trace`` is a
-    dict, each layer's output is stored in it under its name."""
+    gamma, beta, w, b.  Returns the video [3, T', 2H', 2W'].  If ``trace`` is a
+    dict, each layer's output is stored in it under its name.
+
+    temporal=True adds the temporal 2x upsample (temporal_upsample2x) after the
+    upsample convs of the first two stages, so the video has 4T - 3 frames
+    (4T for a continuing chunk, first_chunk=False) instead of T.  Which two of
+    the three upsamplings carry it is a reading: the pages give the frame
+    count, not the place."""
     h = causal_conv3d(z, *params["conv_in"], threads=threads)
     if trace is not None:
         trace["conv_in"] = h
@@ -188,6 +215,8 @@ def trunk(z, params, threads: int | None = None, trace: dict | None = None):
                 trace[f"s{s}.b{r}"] = h
         if st["up"] is not None:
             h = upsample_conv(h, *st["up"], threads=threads)
+            if temporal and s < 2:
+                h = temporal_upsample2x(h, first_chunk)
             if trace is not None:
                 trace[f"s{s}.up"] = h
     hp = params["head"]

@@ -270,10 +270,97 @@ def check_resblock_identity(O):
     assert np.array_equal(O.resblock(x, p), x)
 
 
+# ------------------------------------------------------ temporal upsample
+def load_temporal_golden():
+    src, frames = [], []
+    for line in open(os.path.join(GOLDEN, "temporal_upsample_hand.txt")):
+        f = line.split()
+        if not f or f[0].startswith("#"):
+            continue
+        if f[0] in ("first", "next"):
+            src.append((f[0] == "first", int(f[1]), [int(v) for v in f[2:]]))
+        elif f[0] == "frames":
+            frames.append((int(f[1]), int(f[2])))
+    return src, frames
+
+
+def check_temporal_golden(O):
+    """Hand-listed source frames: frame index t carried in the data itself."""
+    src, _ = load_temporal_golden()
+    for first, T, want in src:
+        x = np.arange(T, dtype=np.float64).reshape(1, T, 1, 1) * np.ones((2, T, 2, 3))
+        y = O.temporal_upsample2x(x, first_chunk=first)
+        assert y.shape == (2, len(want), 2, 3)
+        assert np.array_equal(y[0, :, 0, 0], np.array(want, dtype=np.float64))
+        assert np.array_equal(y, y[:1].repeat(2, 0))    # every channel and pixel alike
+
+
+def check_temporal_library(O):
+    """torch.repeat_interleave on the time axis, less the first copy of frame 0
+    for a decode's first chunk; streaming: chunk by chunk equals all at once."""
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((3, 5, 2, 4))
+    rep = torch.repeat_interleave(torch.from_numpy(x), 2, dim=1).numpy()
+    assert np.array_equal(O.temporal_upsample2x(x, first_chunk=True), rep[:, 1:])
+    assert np.array_equal(O.temporal_upsample2x(x, first_chunk=False), rep)
+    parts = [O.temporal_upsample2x(x[:, :2], True), O.temporal_upsample2x(x[:, 2:], False)]
+    assert np.array_equal(np.concatenate(parts, 1), O.temporal_upsample2x(x, True))
+
+
+def check_temporal_trunk_frames(O, synth):
+    """The trunk with temporal upsampling: 4T - 3 frames (the pages' count,
+    tests/golden/temporal_upsample_hand.txt), the first frame equal to the
+    trunk without it at T = 1, and causal in upsampled time: changing latent
+    frame t >= 1 leaves video frames before 4t - 3 unchanged and changes frame
+    4t - 3."""
+    _, frames = load_temporal_golden()
+    for T, n in frames:
+        if T <= 4:
+            z, params = synth.trunk_input(T=T, H=2, W=2, widths=(8, 8, 8, 8), zc=4, seed=T)
+            assert O.trunk(z, params, temporal=True).shape[1] == n
+    z, params = synth.trunk_input(T=1, H=2, W=3, widths=(8, 8, 8, 8), zc=4, seed=6)
+    assert np.array_equal(O.trunk(z, params, temporal=True), O.trunk(z, params))
+    z, params = synth.trunk_input(T=3, H=2, W=2, widths=(8, 8, 8, 8), zc=4, seed=7)
+    v0 = O.trunk(z, params, temporal=True)
+    for t in (1, 2):
+        z2 = z.clone()
+        z2[:, t] += 1.0
+        v1 = O.trunk(z2, params, temporal=True)
+        assert np.array_equal(v0[:, :4 * t - 3], v1[:, :4 * t - 3])
+        assert not np.allclose(v0[:, 4 * t - 3], v1[:, 4 * t - 3])
+
+
+def torch_trunk_temporal(z, params):
+    """The trunk with temporal upsampling from library routines (float64, CPU):
+    repeat_interleave in time after the first two upsample convs."""
+    def conv(v, w, b):
+        return torch.from_numpy(torch_causal_conv(v.numpy(), w.double().numpy(), b.double().numpy()))
+    h = conv(z.double(), *params["conv_in"])
+    for s, st in enumerate(params["stages"]):
+        for bp in st["blocks"]:
+            h = torch.from_numpy(torch_resblock(h, bp))
+        if st["up"] is not None:
+            h = conv(F.interpolate(h, scale_factor=2, mode="nearest"), *st["up"])
+            if s < 2:
+                h = torch.repeat_interleave(h, 2, dim=1)[:, 1:]
+    hp = params["head"]
+    C = h.shape[0]
+    a = F.silu(F.normalize(h, dim=0, eps=1e-12) * math.sqrt(C) * hp["gamma"].double().view(-1, 1, 1, 1)
+               + hp["beta"].double().view(-1, 1, 1, 1))
+    o = conv(a, hp["w"], hp["b"])
+    return F.pixel_shuffle(o.permute(1, 0, 2, 3), 2).permute(1, 0, 2, 3).numpy()
+
+
+def check_trunk_temporal_library(O, synth):
+    z, params = synth.trunk_input(T=3, H=2, W=3, widths=(16, 16, 8, 8), zc=6, seed=8)
+    np.testing.assert_allclose(O.trunk(z, params, temporal=True), torch_trunk_temporal(z, params),
+                               rtol=1e-9, atol=1e-9)
+
+
 ALL_CHECKS = [check_norm_golden, check_norm_unit_rms, check_norm_scale_invariance,
               check_norm_library, check_silu_limits, check_conv_golden, check_conv_library,
               check_conv_brute, check_conv_invariants, check_upsample, check_pixel_shuffle,
-              check_resblock_identity]
+              check_resblock_identity, check_temporal_golden, check_temporal_library]
 
 
 def torch_trunk(z, params):

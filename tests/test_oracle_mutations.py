@@ -17,7 +17,8 @@ from video_diffusion_vae_b200 import synth
 
 def _ns(**over):
     d = {k: getattr(O, k) for k in ("silu", "norm_silu", "causal_conv3d", "causal_conv3d_at",
-                                    "upsample_nearest2x", "pixel_shuffle2x2", "resblock")}
+                                    "upsample_nearest2x", "pixel_shuffle2x2", "resblock",
+                                    "temporal_upsample2x")}
     d.update(over)
     return types.SimpleNamespace(**d)
 
@@ -195,3 +196,46 @@ def test_trunk_rebuild_without_mistake_passes():
 @pytest.mark.parametrize("name", sorted(TRUNK_MUTANTS))
 def test_pins_catch_trunk_mutant(name):
     assert _trunk_fails(**TRUNK_MUTANTS[name]), f"the trunk pin passed planted mistake {name}"
+
+
+# ------------------------------------------------- the temporal upsample
+def temporal_first_doubled(x, first_chunk=True):
+    return O.temporal_upsample2x(x, first_chunk=False)
+
+
+def temporal_last_once(x, first_chunk=True):
+    # keeps the last frame once instead of the first
+    y = O.temporal_upsample2x(x, first_chunk=False)
+    return y[:, :-1]
+
+
+def temporal_blocked(x, first_chunk=True):
+    # all copies of the first half, then all of the second: a tiled repeat
+    y = O.temporal_upsample2x(x, first_chunk)
+    return np.concatenate([y[:, 0::2], y[:, 1::2]], axis=1)
+
+
+@pytest.mark.parametrize("mutant", [temporal_first_doubled, temporal_last_once, temporal_blocked])
+def test_pins_catch_temporal_mutant(mutant):
+    assert _fails(_ns(temporal_upsample2x=mutant))
+
+
+def test_trunk_temporal_pin_catches_placement_and_count():
+    """The library-built trunk pins the composition: the temporal step after
+    the last upsample conv instead of the first, or a single step, fails."""
+    def trunk_wrong(z, params, threads=None, temporal=False, first_chunk=True, stages=(1, 2)):
+        h = O.causal_conv3d(z, *params["conv_in"])
+        for s, st in enumerate(params["stages"]):
+            for bp in st["blocks"]:
+                h = O.resblock(h, bp)
+            if st["up"] is not None:
+                h = O.upsample_conv(h, *st["up"])
+                if temporal and s in stages:
+                    h = O.temporal_upsample2x(h, first_chunk)
+        hp = params["head"]
+        return O.head(h, hp["gamma"], hp["beta"], hp["w"], hp["b"])
+    for stages in [(1, 2), (0,)]:
+        ns = types.SimpleNamespace(trunk=lambda z, p, threads=None, temporal=False, first_chunk=True,
+                                   st=stages: trunk_wrong(z, p, threads, temporal, first_chunk, st))
+        with pytest.raises(AssertionError):
+            P.check_trunk_temporal_library(ns, synth)

@@ -18,3 +18,11 @@ def test_resblock_against_library():
 
 def test_trunk_against_library():
     P.check_trunk_library(O, synth)
+
+
+def test_trunk_temporal_frames_and_causality():
+    P.check_temporal_trunk_frames(O, synth)
+
+
+def test_trunk_temporal_against_library():
+    P.check_trunk_temporal_library(O, synth)
