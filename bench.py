@@ -45,12 +45,13 @@ L2_FLUSH_BYTES = 512 << 20
 
 
 # ------------------------------------------------------------------ workload
-def trunk_layers(T=T, H=H, W=W, widths=WIDTHS, zc=ZC, executed=False):
+def trunk_layers(T=T, H=H, W=W, widths=WIDTHS, zc=ZC, executed=False, phase_form=False):
     """The trunk's launches in order with their dense FLOPs (all taps counted;
-    the upsample convs at output resolution with 9 taps).  executed=True gives
-    the MMA FLOPs the kernels actually issue instead: the upsample convs run as
-    four 2x2 phase convs on the low-res input (16/36 of dense), conv_in runs
-    on 48 channels padded to 64, the head on 12 output channels padded to 16."""
+    the upsample convs at output resolution with 9 taps).  phase_form=True
+    counts the upsample convs as four 2x2 phase convs on the low-res input
+    (16/36 of dense: the least exact work).  executed=True gives the MMA FLOPs
+    the kernels actually issue: the phase form, conv_in on 48 channels padded
+    to 64, the head on 12 output channels padded to 16."""
     layers = [("layout", 0.0)]
     v = T * H * W
     layers.append(("conv_in", 2.0 * v * widths[0] * (64 if executed else zc) * 27))
@@ -60,7 +61,8 @@ def trunk_layers(T=T, H=H, W=W, widths=WIDTHS, zc=ZC, executed=False):
             layers.append((f"s{s}.b{b}.conv1", 2.0 * vs * c * c * 27))
             layers.append((f"s{s}.b{b}.conv2", 2.0 * vs * c * c * 27))
         if s + 1 < len(widths):
-            up = 2.0 * vs * widths[s + 1] * c * 16 if executed else 2.0 * (4 * vs) * widths[s + 1] * c * 9
+            up = 2.0 * vs * widths[s + 1] * c * 16 if (executed or phase_form) \
+                else 2.0 * (4 * vs) * widths[s + 1] * c * 9
             layers.append((f"s{s}.up", up))
     v3 = v * 4 ** (len(widths) - 1)
     layers.append(("head", 2.0 * v3 * (16 if executed else 12) * widths[-1] * 27))
@@ -234,37 +236,109 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------- CPU baseline
-def oracle_trunk_sample(h=4, w=6):
-    """Time the CPU oracle on the trunk at latents [1, 48, 4, h, w] (full channel
-    widths) and scale to the full 44 x 78 workload by the dense FLOP ratio."""
+ORACLE_CROP = 16
+
+
+def oracle_layer_sample(crop=ORACLE_CROP, seed=1):
+    """The CPU oracle timed on every distinct layer shape of the full workload.
+
+    Each layer runs on a spatial crop of its own input: crop x crop voxels
+    (crop/2 x crop/2 low-res voxels for the upsample convs, whose output is then
+    crop x crop), all 4 frames, the layer's full channel width.  Its time is
+    scaled by the layer's full output voxels over the crop's (the oracle's
+    loops visit every tap of every output voxel, padded or not, so its work per
+    output voxel does not depend on the position) and the layers are summed:
+    conv_in, one residual block per stage (x 2 blocks), the three upsample
+    convs and the head (norm_out + SiLU + conv + pixel shuffle).
+    Returns (frames/s, seconds of oracle work, threads, per-layer detail)."""
+    import torch
     from oracle import oracle as O
     from video_diffusion_vae_b200 import synth
-    z, params = synth.trunk_input(T=T, H=h, W=w, seed=1)
-    t0 = time.perf_counter()
-    O.trunk(z, params)
-    dt = time.perf_counter() - t0
-    f_sample = sum(f for _, f in trunk_layers(T, h, w))
-    f_full = sum(f for _, f in trunk_layers())
-    fps = T / (dt * f_full / f_sample)
-    return fps, dt, O.nthreads(), f"oracle trunk on latents [1,48,{T},{h},{w}] (full widths), " \
-        f"{dt:.1f} s, scaled by dense FLOPs {f_full / f_sample:.0f}x to [1,48,{T},{H},{W}]"
+    _, params = synth.trunk_input(T=T, H=2, W=2, seed=seed)
+    g = torch.Generator().manual_seed(seed)
+    c, ch = crop, crop // 2
+    full_t, spent, detail = 0.0, 0.0, {}
+
+    def run(name, fn, full_vox, crop_vox, count=1):
+        nonlocal full_t, spent
+        t0 = time.perf_counter()
+        fn()
+        dt = time.perf_counter() - t0
+        spent += dt
+        full_t += dt * full_vox / crop_vox * count
+        detail[name] = round(dt * full_vox / crop_vox * count, 2)
+
+    z = synth.normal(g, (ZC, T, c, c))
+    run("conv_in", lambda: O.causal_conv3d(z, *params["conv_in"]), H * W, c * c)
+    Hs, Ws = H, W
+    for s, st in enumerate(params["stages"]):
+        Cs = WIDTHS[s]
+        x = synth.normal(g, (Cs, T, c, c))
+        run(f"s{s}.resblock x2", lambda: O.resblock(x, st["blocks"][0]), Hs * Ws, c * c, 2)
+        if st["up"] is not None:
+            xl = synth.normal(g, (Cs, T, ch, ch))
+            run(f"s{s}.up", lambda: O.upsample_conv(xl, *st["up"]), Hs * Ws, ch * ch)
+            Hs, Ws = 2 * Hs, 2 * Ws
+    hp = params["head"]
+    xh = synth.normal(g, (WIDTHS[-1], T, c, c))
+    run("head", lambda: O.head(xh, hp["gamma"], hp["beta"], hp["w"], hp["b"]), Hs * Ws, c * c)
+    return T / full_t, spent, O.nthreads(), detail
+
+
+def oracle_sample_text(crop, spent, reps):
+    return (f"oracle (fp64 C, all host threads) on each distinct layer shape of the workload: "
+            f"conv_in, one res block per stage, the 3 upsample convs and the head, each on a "
+            f"{crop}x{crop}-voxel spatial crop of its input (4 frames, full channel width), "
+            f"scaled per layer by full/crop output voxels and summed; {reps} sample(s), "
+            f"{spent:.1f} s of oracle work")
+
+
+def bench_config(world):
+    """The `config` object of the JSON line (both arms print the same one)."""
+    return {"workload": WORKLOAD,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "flushed before every timed step, outside the step events (512 MiB written, "
+                  "then read back: no dirty line of the flush left)",
+            "trunk_dense_tflop_per_step": sum(f for _, f in trunk_layers()) / 1e12}
+
+
+def cpu_baseline(reps=3):
+    """Median of `reps` layer-shape samples (about 5 s each on 16 host threads)."""
+    vals, spent, cores, detail = [], 0.0, 1, None
+    for _ in range(reps):
+        fps, dt, cores, detail = oracle_layer_sample()
+        vals.append(fps)
+        spent += dt
+    v = statistics.median(vals)
+    return {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": oracle_sample_text(ORACLE_CROP, spent, reps),
+            "layer_s_full_size": detail, "full_step_s": T / v}
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle, as it stands, on the host cores.  One
+    step is one layer-shape sample of the workload (oracle_layer_sample), so
+    `ms_per_step` is the sample's own duration; `value` is the full workload's
+    frames/s that the sample measures (median over the timed steps)."""
     if rank != 0:
         return 0
-    vals = []
+    vals, secs, cores, spent = [], [], 1, 0.0
     for i in range(args.warmup + args.steps):
-        fps, dt, cores, sample = oracle_trunk_sample(2, 3)
+        fps, dt, cores, _ = oracle_layer_sample()
         if i >= args.warmup:
             vals.append(fps)
+            secs.append(dt)
+            spent += dt
     v = statistics.median(vals)
+    sample = oracle_sample_text(ORACLE_CROP, spent, args.steps)
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": T / v * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(secs) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample": sample},
+        "data": "synthetic (seeded N(0,1) inputs, random weights with the trunk's shapes)",
+        "config": bench_config(world),
+        "step": "one layer-shape sample of the workload (see cpu_baseline.sample); "
+                f"the full workload's step is {T / v:.0f} s at this rate",
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -489,16 +563,25 @@ def main():
         B.decode_trunk(zd, tr, out=video, workspace=ws, events=ev[i])
     torch.cuda.synchronize()
 
-    # per-launch durations -> the dominant kernel (tensor-core conv) and shares
+    # per-launch durations -> the dominant kernel's (the tensor-core conv's)
+    # share of a step; its time in the timed steps is that share of the timed
+    # step (the events pass only apportions the step among its launches)
     per_layer = [[ev[i][2 * j].elapsed_time(ev[i][2 * j + 1]) for j in range(nl)] for i in range(args.steps)]
     conv_idx = [j for j, (name, _) in enumerate(layers) if name != "layout"]
-    conv_ms = statistics.mean(sum(per_layer[i][j] for j in conv_idx) for i in range(args.steps))
+    ev_conv_ms = statistics.mean(sum(per_layer[i][j] for j in conv_idx) for i in range(args.steps))
+    ev_step_ms = statistics.mean(sum(per_layer[i]) for i in range(args.steps))
+    conv_share = ev_conv_ms / ev_step_ms
+    step_ms_timed = total_ms / args.steps            # this rank's timed step
+    conv_launch_ms = conv_share * step_ms_timed / len(conv_idx)
     conv_flops = sum(layers[j][1] for j in conv_idx)
     exec_layers = trunk_layers(executed=True)
+    phase_layers = trunk_layers(phase_form=True)
     conv_flops_exec = sum(exec_layers[j][1] for j in conv_idx)
-    conv_launch_ms = conv_ms / len(conv_idx)
-    achieved = conv_flops / len(conv_idx) / (conv_launch_ms * 1e-3) / 1e12
-    achieved_exec = conv_flops_exec / len(conv_idx) / (conv_launch_ms * 1e-3) / 1e12
+    conv_flops_phase = sum(phase_layers[j][1] for j in conv_idx)
+    per_launch_s = conv_launch_ms * 1e-3
+    achieved = conv_flops / len(conv_idx) / per_launch_s / 1e12
+    achieved_phase = conv_flops_phase / len(conv_idx) / per_launch_s / 1e12
+    achieved_exec = conv_flops_exec / len(conv_idx) / per_launch_s / 1e12
     layer_ms = {layers[j][0]: statistics.mean(per_layer[i][j] for i in range(args.steps)) for j in range(nl)}
 
     # ---- e2e: every step copies its latents from pinned host memory and its
@@ -555,33 +638,37 @@ def main():
         comp = components(peaks, flush)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        fps, dt, cores, sample = oracle_trunk_sample()
-        cpu = {"value": fps, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+        cpu = cpu_baseline()
 
     if rank == 0:
-        peak_t = peaks["bf16_tflops_sustained"]
+        peak_t = peaks["bf16_tflops"]
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) latents, random weights with the trunk's shapes)",
-            "config": {"workload": WORKLOAD,
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "flushed before every timed step, outside the step events (512 MiB written, then read back: no dirty line of the flush left)",
-                       "trunk_dense_tflop_per_step": sum(f for _, f in layers) / 1e12},
+            "config": bench_config(world),
             "tflops": sum(f for _, f in layers) * args.steps / (total_ms * 1e-3) / 1e12,
             "roofline": {"bound": "tensor", "kernel": "conv_tc_kernel (all 21 conv launches of a step)",
                          "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
-                         "frac": achieved / peak_t, "peak_kind": f"{peak_kind} bf16 sustained",
-                         "frac_of_burst": achieved / peaks["bf16_tflops"], "frac_of_2250": achieved / 2250.0,
+                         "frac": achieved / peak_t,
+                         "peak_kind": f"{peak_kind} bf16 burst (sub-millisecond launches)",
+                         "traffic": conv_traffic(), "traffic_unit": "bytes per launch (mean of the 21)",
                          "flops_per_launch": conv_flops / len(conv_idx),
+                         "flop_count": "dense: every tap of the causal convs, the upsample convs "
+                                       "at output resolution with 9 taps",
+                         "achieved_phase_form": achieved_phase,
+                         "frac_phase_form": achieved_phase / peak_t,
                          "achieved_executed": achieved_exec,
                          "frac_executed": achieved_exec / peak_t,
-                         "traffic": conv_traffic(), "traffic_unit": "bytes per launch (mean of the 21)",
+                         "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                         "frac_of_2250": achieved / 2250.0,
                          "launch_ms": conv_launch_ms,
-                         "launch_timing": "CUDA events around each launch, a separate pass of the same "
-                                          "steps after the timed one",
-                         "conv_share_of_step": conv_ms / statistics.mean(step_ms)},
+                         "conv_share_of_step": conv_share,
+                         "launch_timing": "the convs' share of a step, from CUDA events around "
+                                          "every launch in a second pass of the same steps, times "
+                                          "the timed step's duration",
+                         "events_pass_step_ms": ev_step_ms},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": zh.numel() * 2,
                     "d2h_bytes_per_step": vh[0].numel() * 2,

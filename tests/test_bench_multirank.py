@@ -9,6 +9,8 @@ import pytest
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
+from tests.ports import free_port
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
@@ -26,7 +28,7 @@ def _rank(rank, world, port, q):
 def test_max_over_ranks_gloo():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = 29611
+    port = free_port()
     ps = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
     for p in ps:
         p.start()
@@ -49,7 +51,7 @@ def test_single_rank_identity():
 @pytest.mark.slow
 def test_reference_arm_under_torchrun():
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
-           "--master-addr", "127.0.0.1", "--master-port", "29612", os.path.join(ROOT, "bench.py"),
+           "--master-addr", "127.0.0.1", "--master-port", str(free_port()), os.path.join(ROOT, "bench.py"),
            "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0"]
     out = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT)
     assert out.returncode == 0, out.stderr[-2000:]

@@ -84,7 +84,13 @@ def test_conv_full_size_sampled():
     y = B.causal_conv3d(to_cl(x), pk)
     torch.cuda.synchronize()
     yc = y.float().cpu()
-    pts = sample_voxels(4, 88, 156, 48, seed=2)
+    # 512 voxels: corners and edges, the seams of the 8 x 32 CTA tiles (rows
+    # 7 | 8, columns 31 | 32), the two 4-row MMA sub-tiles of a tile (rows
+    # 3 | 4), the ragged last tile column (128..155), every frame, and
+    # uniformly drawn voxels
+    seams = {(t, h, c) for t in range(4) for h in (3, 4, 7, 8, 83, 84, 87)
+             for c in (31, 32, 127, 128, 155)}
+    pts = sorted(set(sample_voxels(4, 88, 156, 512 - len(seams), seed=2)) | seams)
     got = np.stack([yc[t, h, ww].double().numpy() for (t, h, ww) in pts], 1)
     ref = np.stack([O.causal_conv3d_at(x, w, b, t, h, ww) for (t, h, ww) in pts], 1)
     assert_close(got, ref, torch.bfloat16, "512->512 full size sampled")

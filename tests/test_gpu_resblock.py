@@ -49,7 +49,12 @@ def test_resblock_full_size_sampled(cout):
     y = B.resblock(to_cl(x), blk)
     torch.cuda.synchronize()
     yc = y.float().cpu()
-    pts = sample_voxels(4, 176, 312, 12, seed=3)
+    # 256 voxels: corners and edges, the seams of the 16 x 16 CTA tiles (rows
+    # 15 | 16, columns 15 | 16), the two 8-row MMA sub-tiles of a tile (rows
+    # 7 | 8), the last frame, and uniformly drawn voxels
+    seams = {(t, h, w) for t in (0, 3) for h in (7, 8, 15, 16, 167, 168, 175)
+             for w in (15, 16, 303, 304, 311)}
+    pts = sorted(set(sample_voxels(4, 176, 312, 256 - len(seams), seed=3)) | seams)
     got = np.stack([yc[t, h, w].double().numpy() for (t, h, w) in pts], 1)
     ref = np.stack([resblock_at(x, p, t, h, w) for (t, h, w) in pts], 1)
     assert_close(got, ref, torch.bfloat16, f"res block 256->{cout}")
@@ -144,57 +149,6 @@ def test_trunk_full_size_properties():
     v2 = B.decode_trunk(z2, tr)
     assert torch.equal(v0[:, :, :3], v2[:, :, :3])
     assert not torch.equal(v0[:, :, 3], v2[:, :, 3])
-    assert B.device_error() == 0
-
-
-def test_trunk_full_size_vs_standalone_entry_points():
-    """The trunk at full size (latents [1, 48, 4, 44, 78]), every output element:
-    the fused trunk against the same decoder composed from the standalone entry
-    points (causal conv, res block, upsample conv, norm-SiLU prologue), each
-    checked against the oracle above.  This covers what only full-size layers run (several tiles per CTA,
-    the early accumulator release, wave-balanced tile shapes).  The paths round
-    differently (fp32 residual stream and fused norms vs bf16 between calls),
-    so the bound is the sum of the two paths' bounds against the oracle:
-    rel-L2 <= 2e-2 and max |diff| <= 1e-1 x std."""
-    T, H, W = 4, 44, 78
-    z, params = synth.trunk_input(T=T, H=H, W=W, seed=0)
-    tr = B.PackedTrunk(params)
-    video = B.decode_trunk(z[None].cuda().bfloat16().contiguous(), tr)
-
-    dev = torch.device("cuda")
-    # conv_in: the standalone bf16 conv takes Cin in multiples of 64 -> zero channels
-    w, b = params["conv_in"]
-    wp = torch.zeros(w.shape[0], 64, *w.shape[2:])
-    wp[:, :48] = w
-    x = torch.zeros(T, H, W, 64)
-    x[..., :48] = z.permute(1, 2, 3, 0)
-    h = B.causal_conv3d(x.to(dev, torch.bfloat16).contiguous(),
-                        B.prepack_conv(wp.to(dev, torch.bfloat16), b.to(dev)))
-    for st in params["stages"]:
-        for bp in st["blocks"]:
-            h = B.resblock(h, B.PackedResBlock(bp))
-        if st["up"] is not None:
-            uw, ub = st["up"]
-            h = B.upsample_conv(h, B.prepack_upsample_conv(uw.to(dev, torch.bfloat16), ub.to(dev)))
-    hp = params["head"]
-    # head: 12 output channels padded to 16 with zero weights; norm_out + SiLU as the prologue
-    hw = torch.zeros(16, *hp["w"].shape[1:])
-    hw[:12] = hp["w"]
-    hb = torch.zeros(16)
-    hb[:12] = hp["b"]
-    y = B.causal_conv3d(h, B.prepack_conv(hw.to(dev, torch.bfloat16), hb.to(dev)),
-                        norm=(hp["gamma"].to(dev), hp["beta"].to(dev)))
-    Tn, Hn, Wn = y.shape[:3]
-    # 2x2 pixel shuffle: video[c, t, 2h+i, 2w+j] = y[t, h, w, 4c + 2i + j]
-    ref = y[..., :12].float().reshape(Tn, Hn, Wn, 3, 2, 2).permute(3, 0, 1, 4, 2, 5)
-    ref = ref.reshape(3, Tn, 2 * Hn, 2 * Wn)
-    got = video[0].float()
-    assert got.shape == ref.shape == (3, 4, 704, 1248)
-    diff = (got - ref).double()
-    rel = (diff.norm() / ref.double().norm()).item()
-    mx = (diff.abs().max() / ref.double().std()).item()
-    assert rel <= 2e-2, f"rel L2 {rel:.3e}"
-    assert mx <= 1e-1, f"max |diff| / std {mx:.3e}"
     assert B.device_error() == 0
 
 

@@ -13,6 +13,7 @@ import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
+from tests.ports import free_port
 from video_diffusion_vae_b200 import shard
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -130,14 +131,62 @@ def _run(world, port, H, norm_after_exchange=False):
     return dict(q.get(timeout=10) for _ in range(world))
 
 
-@pytest.mark.parametrize("world,port", [(2, 29631), (3, 29632)])
-def test_row_split_trunk_equals_whole(world, port):
-    got = _run(world, port, H=5)
+@pytest.mark.parametrize("world", [2, 3])
+def test_row_split_trunk_equals_whole(world):
+    got = _run(world, free_port(), H=5)
     assert all(got.values()), got
 
 
 def test_row_split_needs_the_activated_halo():
     """Exchanging the raw tensor and normalising the halo rows as well gives
     the wrong border (SiLU(beta) where the frame pads with zeros)."""
-    got = _run(2, 29633, H=4, norm_after_exchange=True)
+    got = _run(2, free_port(), H=4, norm_after_exchange=True)
     assert not all(got.values())
+
+
+# ------------------------------------------------- a subgroup of the ranks
+def _sub_rank(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        sub = dist.new_group([1, 2])              # every rank creates it
+        if rank in (1, 2):
+            r, n = dist.get_rank(sub), dist.get_world_size(sub)
+            parts = shard.partition(6, n)
+            r0, r1 = parts[r]
+            full = torch.arange(6 * 4, dtype=torch.float32).view(1, 6, 4)   # [T, rows, W]
+            ext = shard.with_halo(full[:, r0:r1].clone(), 1)
+            shard.exchange_halo(ext, r, n, 1, group=sub)
+            want_top = full[:, r0 - 1] if r0 > 0 else torch.zeros(1, 4)
+            want_bot = full[:, r1] if r1 < 6 else torch.zeros(1, 4)
+            ok = torch.equal(ext[:, 0], want_top) and torch.equal(ext[:, -1], want_bot)
+            got = shard.gather_rows(full[:, r0:r1], parts, 1, r, n, 1, group=sub)
+            ok = ok and (torch.equal(got, full) if r == 0 else got is None)
+            q.put((rank, ok))
+        else:
+            q.put((rank, True))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_halo_and_gather_on_a_subgroup():
+    """Ranks {1, 2} of 3 as their own group: group rank 0 is global rank 1, so
+    peers must be addressed by their global ranks."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    ps = [ctx.Process(target=_sub_rank, args=(r, 3, port, q)) for r in range(3)]
+    for p in ps:
+        p.start()
+    for p in ps:
+        p.join(120)
+    for p in ps:
+        if p.is_alive():
+            p.terminate()
+            p.join(10)
+    assert all(p.exitcode == 0 for p in ps), [p.exitcode for p in ps]
+    got = dict(q.get(timeout=10) for _ in range(3))
+    assert all(got.values()), got

@@ -59,14 +59,20 @@ def with_halo(x: torch.Tensor, row_dim: int) -> torch.Tensor:
     return out
 
 
+def _peer(group, r: int) -> int:
+    """The global rank of rank r of `group` (torch addresses peers globally)."""
+    return r if group is None else dist.get_global_rank(group, r)
+
+
 def exchange_halo(x_ext: torch.Tensor, rank: int, world: int, row_dim: int, group=None) -> None:
     """Fill the halo rows of x_ext in place.
 
     x_ext holds, along row_dim, one halo row, the rank's own rows, one halo row.
     Row 0 receives the last own row of rank - 1 (zeros on rank 0); the last row
-    receives the first own row of rank + 1 (zeros on the last rank).  Every
-    rank of the group must call it (ranks with one neighbour exchange with it
-    alone)."""
+    receives the first own row of rank + 1 (zeros on the last rank).  `rank`
+    and `world` are this process's rank in `group` and the group's size (the
+    default group when None).  Every rank of the group must call it (ranks
+    with one neighbour exchange with it alone)."""
     n = x_ext.shape[row_dim]
     if n < 3:
         raise ValueError("x_ext needs at least one own row between the two halo rows")
@@ -76,11 +82,11 @@ def exchange_halo(x_ext: torch.Tensor, rank: int, world: int, row_dim: int, grou
     bottom = torch.zeros_like(first)
     ops = []
     if rank > 0:
-        ops.append(dist.P2POp(dist.isend, first, rank - 1, group))
-        ops.append(dist.P2POp(dist.irecv, top, rank - 1, group))
+        ops.append(dist.P2POp(dist.isend, first, _peer(group, rank - 1), group))
+        ops.append(dist.P2POp(dist.irecv, top, _peer(group, rank - 1), group))
     if rank < world - 1:
-        ops.append(dist.P2POp(dist.isend, last, rank + 1, group))
-        ops.append(dist.P2POp(dist.irecv, bottom, rank + 1, group))
+        ops.append(dist.P2POp(dist.isend, last, _peer(group, rank + 1), group))
+        ops.append(dist.P2POp(dist.irecv, bottom, _peer(group, rank + 1), group))
     if ops:
         for req in dist.batch_isend_irecv(ops):
             req.wait()
@@ -90,15 +96,18 @@ def exchange_halo(x_ext: torch.Tensor, rank: int, world: int, row_dim: int, grou
 
 def gather_rows(mine: torch.Tensor, parts: list[tuple[int, int]], scale: int, rank: int,
                 world: int, row_dim: int, group=None):
-    """Rank 0 receives every rank's rows (`mine`: this rank's rows at `scale`
-    times the latent resolution, along row_dim) and returns the whole tensor;
-    the other ranks send theirs and return None.  Every rank of the group must
-    call it."""
+    """Rank 0 of the group receives every rank's rows (`mine`: this rank's rows
+    at `scale` times the latent resolution, along row_dim) and returns the
+    whole tensor; the other ranks send theirs and return None.  Every rank of
+    the group must call it.  Rank 0 sizes each receive buffer from its own
+    tensor, so every rank's `mine` must have rank 0's dtype and rank 0's shape
+    apart from row_dim (whose length must be the rank's row count: checked).
+    `rank` and `world` are this process's rank in `group` and its size."""
     r0, r1 = rows_at(parts[rank], scale)
     if mine.shape[row_dim] != r1 - r0:
         raise ValueError(f"rank {rank} holds {mine.shape[row_dim]} rows, its part has {r1 - r0}")
     if rank != 0:
-        dist.send(mine.contiguous(), 0, group)
+        dist.send(mine.contiguous(), _peer(group, 0), group)
         return None
     pieces = [mine.contiguous()]
     for src in range(1, world):
@@ -106,6 +115,6 @@ def gather_rows(mine: torch.Tensor, parts: list[tuple[int, int]], scale: int, ra
         shape = list(mine.shape)
         shape[row_dim] = b - a
         buf = mine.new_empty(shape)
-        dist.recv(buf, src, group)
+        dist.recv(buf, _peer(group, src), group)
         pieces.append(buf)
     return torch.cat(pieces, dim=row_dim)
