@@ -9,10 +9,11 @@
  *   - causal 3x3x3 conv3d with bf16 operands and fp32 accumulation (FastVideo
  *     "Wan2.2 VAE decoder (sm_100a, sm_103a)" README, section "Limits");
  *   - the residual block, the nearest-2x upsample + 3x3 conv, and the decoder
- *     trunk from latents [1, 48, T, H, W] to video [1, 3, T, 16H, 16W]
- *     (same README, opening section: 48 latent channels, 16x16 spatial
- *     compression; raw entry points are destination-passing on the current
- *     stream, section "Use").
+ *     trunk from latents [1, 48, T, H, W] to video [1, 3, T, 16H, 16W], or,
+ *     with the decoder's temporal upsampling, [1, 3, 4T - 3, 16H, 16W]
+ *     (same README, opening section: 48 latent channels, 16x16 spatial and
+ *     4x temporal compression; raw entry points are destination-passing on
+ *     the current stream, section "Use").
  *
  * Conventions shared by every entry point:
  *   - Memory: every pointer argument named as a tensor is a DEVICE pointer owned
@@ -253,6 +254,36 @@ WVAE_API wvae_status wvae_decode_trunk_chunk(const void* const* packed, const fl
                                     const int* widths, wvae_dtype dtype, void* workspace,
                                     size_t ws_bytes, void* cache, size_t cache_bytes,
                                     int continue_chunk, wvae_stream_t stream);
+
+/* ----------------------------------------- video decode with 4T - 3 frames
+ * The trunk with the decoder's 4x temporal expansion: latents [1][48][T][H][W]
+ * decode to the video [1][3][4T - 3][16H][16W] (FastVideo README, opening
+ * section: 4x temporal compression, video [1, 3, 4T - 3, 704, 1248]).  The
+ * pages give the frame count, not the layer that makes it; this library
+ * reads it as a nearest 2x step in time after the upsample convs of stages 0
+ * and 1: the decode's first frame stays one frame, every later frame becomes
+ * two consecutive frames (T -> 2T - 1, twice: 4T - 3).  The step rides in
+ * those upsample convs' epilogues (each output written to both of its
+ * frames), so it costs no launch; stages 1, 2 and 3 run on 2T - 1, 4T - 3
+ * and 4T - 3 frames.
+ * Arguments as wvae_decode_trunk_chunk, except:
+ *   video: [1][3][wvae_decode_video_frames(T, continue_chunk)][16H][16W].
+ *   workspace: wvae_decode_video_workspace_bytes(T, H, W, widths) bytes.
+ *   cache: NULL for a whole decode (continue_chunk must then be 0); else as
+ *     in wvae_decode_trunk_chunk (wvae_decode_trunk_cache_bytes, T >= 2).  A
+ *     continuing chunk holds no first frame, so all of its frames double and
+ *     it yields 4T frames; chunk by chunk the video equals the whole decode's.
+ * wvae_decode_video_frames returns 4T - 3 (continue_chunk == 0) or 4T, 0 for
+ * T < 1.  Returns WVAE_ERR_INVALID_ARG for continue_chunk without a cache,
+ * as wvae_decode_trunk_chunk otherwise.
+ */
+WVAE_API int wvae_decode_video_frames(int T, int continue_chunk);
+WVAE_API size_t wvae_decode_video_workspace_bytes(int T, int H, int W, const int* widths);
+WVAE_API wvae_status wvae_decode_video(const void* const* packed, const float* const* norms,
+                                       const void* z, void* video, int T, int H, int W,
+                                       const int* widths, wvae_dtype dtype, void* workspace,
+                                       size_t ws_bytes, void* cache, size_t cache_bytes,
+                                       int continue_chunk, wvae_stream_t stream);
 
 /* ------------------------------------------------- res block, no allocation
  * (No counterpart on the pages: this is a convenience of this library.)

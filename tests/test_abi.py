@@ -20,7 +20,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     declared = B.header_symbols()
-    assert len(declared) == 22
+    assert len(declared) == 25
     out = subprocess.check_output(["nm", "-D", "--defined-only", B.LIB_PATH], text=True)
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
     missing = [s for s in declared if s not in exported]
@@ -170,3 +170,20 @@ def test_trunk_cache_bytes_and_chunk_validation():
     assert lib.wvae_decode_trunk_chunk(P, N, A, A, 4, H, W, w, B.BF16, A, 1 << 40, NULL, 0, 0,
                                        NULL) == 1
 
+
+
+def test_video_decode_frames_and_validation():
+    """4T - 3 frames (4T for a continuing chunk); a continuing chunk without a
+    cache, T < 2 with a cache, and a short workspace are refused on the host."""
+    lib = B.load()
+    assert [lib.wvae_decode_video_frames(T, 0) for T in (1, 2, 4, 49)] == [1, 5, 13, 193]
+    assert lib.wvae_decode_video_frames(4, 1) == 16 and lib.wvae_decode_video_frames(0, 0) == 0
+    w = (ctypes.c_int * 4)(512, 512, 256, 128)
+    H, W = 44, 78
+    ws = lib.wvae_decode_video_workspace_bytes(4, H, W, w)
+    assert ws > lib.wvae_decode_trunk_workspace_bytes(4, H, W, w)
+    P = (ctypes.c_void_p * 21)(*([A] * 21))
+    N = (ctypes.c_void_p * 34)(*([A] * 34))
+    assert lib.wvae_decode_video(P, N, A, A, 4, H, W, w, B.BF16, A, ws, NULL, 0, 1, NULL) == 1
+    assert lib.wvae_decode_video(P, N, A, A, 1, H, W, w, B.BF16, A, ws, A, 1 << 40, 0, NULL) == 1
+    assert lib.wvae_decode_video(P, N, A, A, 4, H, W, w, B.BF16, A, 1024, NULL, 0, 0, NULL) == 4

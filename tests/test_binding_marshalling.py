@@ -136,6 +136,23 @@ def test_trunk_and_stream(fake):
     assert [c[1][13] for c in chunk_calls] == [0, 1]   # continue_chunk: first chunk, then carried
 
 
+def test_video_decode_and_stream(fake):
+    """The temporal decode: 4T - 3 frames for a whole decode or a first chunk,
+    4T for a continuing one; no cache for a whole decode."""
+    fake.wvae_decode_video_frames = lambda T, c: 4 * T if c else 4 * T - 3
+    z, params = synth.trunk_input(T=2, H=2, W=3, widths=(64, 64, 64, 64), blocks=2)
+    tr = B.PackedTrunk(params, device="cpu")
+    zd = z[None].bfloat16().contiguous()
+    v = B.decode_video(zd, tr)
+    assert v.shape == (1, 3, 5, 32, 48) and names(fake)[-1] == "wvae_decode_video"
+    assert fake.calls[-1][1][11] is None and fake.calls[-1][1][13] == 0   # cache, continue
+    st = B.VideoStream(tr, 2, 3, device="cpu")
+    a, b = st.decode(zd), st.decode(zd)
+    assert a.shape[2] == 5 and b.shape[2] == 8
+    calls = [c for c in fake.calls if c[0] == "wvae_decode_video"]
+    assert [c[1][13] for c in calls] == [0, 0, 1]
+
+
 def test_caller_workspace_must_be_a_cuda_tensor(fake):
     with pytest.raises(TypeError):
         fake.real_cuda(torch.empty(64, dtype=torch.uint8), "workspace")

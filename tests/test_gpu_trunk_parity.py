@@ -116,3 +116,69 @@ def test_trunk_chunked_decode_vs_oracle(T, H, W, widths, chunks):
     got = torch.cat(parts, dim=2)[0].float().cpu().double().numpy()
     assert_close(got, O.trunk(z, params), torch.bfloat16, f"chunked {chunks}")
     assert B.device_error() == 0
+
+
+# ------------------------------------------- video decode with 4T - 3 frames
+@pytest.mark.parametrize("T,H,W,widths", [
+    (3, 3, 5, (128, 128, 64, 64)),
+    (2, 6, 10, (64, 64, 64, 128)),   # stage 3: 5 frames x 60 tiles of 16 x 16 at 96 x 160
+])
+def test_video_decode_vs_oracle(T, H, W, widths):
+    """The temporal 2x steps ride in the first two upsample convs' epilogues:
+    video [1, 3, 4T - 3, 16H, 16W] against the oracle's decode with them."""
+    z, params = synth.trunk_input(T=T, H=H, W=W, widths=widths, seed=23)
+    tr = B.PackedTrunk(params)
+    v = B.decode_video(z[None].cuda().bfloat16().contiguous(), tr)
+    torch.cuda.synchronize()
+    assert v.shape == (1, 3, 4 * T - 3, 16 * H, 16 * W)
+    ref = O.trunk(z, params, temporal=True)
+    assert_close(v[0].float().cpu().double().numpy(), ref, torch.bfloat16, f"video T={T}")
+    assert B.device_error() == 0
+
+
+@pytest.mark.parametrize("chunks", [(2, 3), (2, 2, 2)])
+def test_video_stream_vs_oracle(chunks):
+    """Chunk by chunk: the first chunk keeps its first frame once (4T - 3
+    frames), later chunks double every frame (4T); together the oracle's
+    whole decode."""
+    T = sum(chunks)
+    z, params = synth.trunk_input(T=T, H=3, W=5, widths=(128, 128, 64, 64), seed=29)
+    tr = B.PackedTrunk(params)
+    zd = z[None].cuda().bfloat16().contiguous()
+    stream = B.VideoStream(tr, 3, 5)
+    parts, t0 = [], 0
+    for i, n in enumerate(chunks):
+        parts.append(stream.decode(zd[:, :, t0:t0 + n].contiguous()))
+        assert parts[-1].shape[2] == (4 * n - 3 if i == 0 else 4 * n)
+        t0 += n
+    torch.cuda.synchronize()
+    got = torch.cat(parts, dim=2)[0].float().cpu().double().numpy()
+    assert_close(got, O.trunk(z, params, temporal=True), torch.bfloat16, f"video chunks {chunks}")
+    assert B.device_error() == 0
+
+
+def test_video_decode_full_size_properties():
+    """Latents [1, 48, 4, 44, 78] -> video [1, 3, 13, 704, 1248]: finite; two
+    chunks of 2 equal the whole decode bit for bit; the first video frame
+    (which sees only latent frame 0 at every stage) is the plain trunk's first
+    frame; changing latent frame 3 leaves video frames 0..8 (before 4*3 - 3)
+    unchanged."""
+    z, params = synth.trunk_input(T=4, H=44, W=78, seed=0)
+    tr = B.PackedTrunk(params)
+    zd = z[None].cuda().bfloat16().contiguous()
+    v = B.decode_video(zd, tr)
+    assert v.shape == (1, 3, 13, 704, 1248)
+    assert torch.isfinite(v.float()).all()
+    stream = B.VideoStream(tr, 44, 78)
+    a = stream.decode(zd[:, :, :2].contiguous())
+    b = stream.decode(zd[:, :, 2:].contiguous())
+    assert torch.equal(torch.cat([a, b], 2), v)
+    plain = B.decode_trunk(zd, tr)
+    rel = ((v[:, :, 0].float() - plain[:, :, 0].float()).norm() / plain[:, :, 0].float().norm()).item()
+    assert rel < 1e-3, rel
+    z2 = zd.clone()
+    z2[:, :, 3] = 0
+    v2 = B.decode_video(z2, tr)
+    assert torch.equal(v[:, :, :9], v2[:, :, :9])
+    assert not torch.equal(v[:, :, 9], v2[:, :, 9])
+    assert B.device_error() == 0

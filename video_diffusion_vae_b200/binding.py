@@ -75,6 +75,10 @@ def load(path: str | None = None):
             "wvae_decode_trunk_cache_bytes": (S, [I, I, ctypes.POINTER(I)]),
             "wvae_decode_trunk_chunk": (I, [ctypes.POINTER(V), ctypes.POINTER(V), V, V, I, I, I,
                                             ctypes.POINTER(I), I, V, S, V, S, I, V]),
+            "wvae_decode_video_frames": (I, [I, I]),
+            "wvae_decode_video_workspace_bytes": (S, [I, I, I, ctypes.POINTER(I)]),
+            "wvae_decode_video": (I, [ctypes.POINTER(V), ctypes.POINTER(V), V, V, I, I, I,
+                                      ctypes.POINTER(I), I, V, S, V, S, I, V]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -330,6 +334,9 @@ class PackedTrunk:
     def cache_bytes(self, H, W):
         return load().wvae_decode_trunk_cache_bytes(H, W, self._widths_arr)
 
+    def video_workspace_bytes(self, T, H, W):
+        return load().wvae_decode_video_workspace_bytes(T, H, W, self._widths_arr)
+
 
 def trunk_launches() -> int:
     return load().wvae_decode_trunk_launches()
@@ -390,6 +397,52 @@ class TrunkStream:
         self.started = True
         return y
 
+
+
+def video_frames(T: int, continue_chunk: bool = False) -> int:
+    """Video frames of a decode with temporal upsampling: 4T - 3, or 4T for a
+    continuing chunk."""
+    return load().wvae_decode_video_frames(int(T), int(continue_chunk))
+
+
+def _decode_video(z, trunk, out, workspace, cache, started):
+    _cuda(z, "z", torch.bfloat16)
+    _, zc, T, H, W = z.shape
+    if zc != 48 or z.shape[0] != 1:
+        raise ValueError("z must be [1, 48, T, H, W]")
+    n = video_frames(T, started)
+    y = torch.empty((1, 3, n, 16 * H, 16 * W), dtype=torch.bfloat16, device=z.device) \
+        if out is None else _cuda(out, "out", torch.bfloat16, (1, 3, n, 16 * H, 16 * W))
+    ws = _ws(workspace, trunk.video_workspace_bytes(T, H, W), z.device)
+    _check("wvae_decode_video", load().wvae_decode_video(
+        trunk._packed_arr, trunk._norm_arr, _ptr(z), _ptr(y), T, H, W, trunk._widths_arr, BF16,
+        _ptr(ws), _nbytes(ws), _ptr(cache), 0 if cache is None else _nbytes(cache), int(started),
+        _stream()))
+    return y
+
+
+def decode_video(z, trunk: PackedTrunk, out=None, workspace=None):
+    """z: latents [1, 48, T, H, W] bf16 (CUDA) -> video [1, 3, 4T - 3, 16H, 16W] bf16:
+    the trunk with the temporal 2x steps after the first two upsample convs."""
+    return _decode_video(z, trunk, out, workspace, None, False)
+
+
+class VideoStream:
+    """Chunked decode with temporal upsampling: the first chunk of T latent
+    frames gives 4T - 3 video frames, each later one 4T; concatenated, they
+    equal decode_video of all the latents."""
+
+    def __init__(self, trunk: PackedTrunk, H, W, device="cuda"):
+        self.trunk, self.H, self.W = trunk, H, W
+        self.cache = _workspace(trunk.cache_bytes(H, W), torch.device(device))
+        self.started = False
+
+    def decode(self, z, out=None, workspace=None):
+        if tuple(z.shape[3:]) != (self.H, self.W):
+            raise ValueError(f"z must be [1, 48, T, {self.H}, {self.W}]")
+        y = _decode_video(z, self.trunk, out, workspace, self.cache, self.started)
+        self.started = True
+        return y
 
 
 class TrunkGraph:

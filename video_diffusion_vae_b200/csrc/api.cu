@@ -145,6 +145,7 @@ struct TcConv {
   const void* packed2 = nullptr;
   int T = 0, H = 0, W = 0;
   int phases = 1;            // 4: upsample-conv phase mode (packed by prepack_upsample)
+  int tdup = 0;              // phase mode: temporal 2x copies of the output (ConvParams::tdup)
   ConvEpilogue ep{};
 };
 
@@ -171,6 +172,7 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   p.KH = a.KH;
   p.KW = a.KW;
   p.phases = a.phases;
+  p.tdup = a.phases == 4 ? a.tdup : 0;
   p.has_cache = a.cache != nullptr;
   // The fused norm needs every output channel of a voxel: one CTA holds them
   // all (BN = Cout) up to 256; at 512 a cluster of two CTAs splits N and swaps
@@ -613,7 +615,8 @@ struct TrunkBuffers {
   size_t total;
 };
 
-TrunkBuffers trunk_buffers(int T, int H, int W, const int* C) {
+// F: frames per stage (T everywhere without temporal upsampling).
+TrunkBuffers trunk_buffers(const int* F, int H, int W, const int* C) {
   TrunkBuffers b;
   size_t off = 0;
   auto take = [&](size_t n) {
@@ -621,10 +624,10 @@ TrunkBuffers trunk_buffers(int T, int H, int W, const int* C) {
     off += round_up_sz(n, 256);
     return o;
   };
-  const size_t v0 = static_cast<size_t>(T) * H * W;
+  const size_t v0 = static_cast<size_t>(F[0]) * H * W;
   size_t max_h = 0, max_act = 0, max_up = 0;
   for (int s = 0; s < 4; ++s) {
-    const size_t vs = v0 << (2 * s);
+    const size_t vs = (static_cast<size_t>(F[s]) * H * W) << (2 * s);
     max_h = std::max(max_h, vs * C[s] * 4);
     max_act = std::max(max_act, vs * C[s] * 2);
     if (s < 3) max_up = std::max(max_up, vs * C[s] * 2);
@@ -685,7 +688,22 @@ size_t wvae_decode_trunk_workspace_bytes(int T, int H, int W, const int* widths)
   const int* C = widths ? widths : kDefaultWidths;
   for (int s = 0; s < 4; ++s)
     if (C[s] < 64) return 0;
-  return trunk_buffers(T, H, W, C).total;
+  const int F[4] = {T, T, T, T};
+  return trunk_buffers(F, H, W, C).total;
+}
+
+int wvae_decode_video_frames(int T, int continue_chunk) {
+  if (T < 1) return 0;
+  return continue_chunk ? 4 * T : 4 * T - 3;
+}
+
+size_t wvae_decode_video_workspace_bytes(int T, int H, int W, const int* widths) {
+  if (T < 1 || H < 1 || W < 1) return 0;
+  const int* C = widths ? widths : kDefaultWidths;
+  for (int s = 0; s < 4; ++s)
+    if (C[s] < 64) return 0;
+  const int F[4] = {T, 2 * T, 4 * T, 4 * T};  // a continuing chunk's counts bound the first's
+  return trunk_buffers(F, H, W, C).total;
 }
 
 namespace {
@@ -698,7 +716,7 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
                               void* video, int T, int H, int W, const int* widths,
                               wvae_dtype dtype, void* workspace, size_t ws_bytes,
                               void* const* events, int n_events, void* cache, size_t cache_bytes,
-                              int continue_chunk, wvae_stream_t stream) {
+                              int continue_chunk, int temporal, wvae_stream_t stream) {
   if (!packed || !norms || !z || !video || !workspace) return WVAE_ERR_INVALID_ARG;
   if (cache != nullptr && T < 2) return WVAE_ERR_INVALID_ARG;  // the cache holds two frames
   if (events != nullptr && n_events < 2 * kTrunkLaunches) return WVAE_ERR_INVALID_ARG;
@@ -714,7 +732,17 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
   for (int i = 0; i < 21; ++i)
     if (!a16(packed[i])) return WVAE_ERR_ALIGNMENT;
   if (!a16(z) || !a16(video) || !a16(workspace)) return WVAE_ERR_ALIGNMENT;
-  const TrunkBuffers B = trunk_buffers(T, H, W, C);
+  if (continue_chunk && cache == nullptr) return WVAE_ERR_INVALID_ARG;
+  // Frames per stage: with temporal upsampling the upsample convs of stages 0
+  // and 1 also double the frames (the decode's first frame once).
+  const bool first = !continue_chunk;
+  int F[4] = {T, T, T, T};
+  if (temporal) {
+    F[1] = first ? 2 * T - 1 : 2 * T;
+    F[2] = first ? 2 * F[1] - 1 : 2 * F[1];
+    F[3] = F[2];
+  }
+  const TrunkBuffers B = trunk_buffers(F, H, W, C);
   if (ws_bytes < B.total) return WVAE_ERR_WORKSPACE;
   const TrunkCaches K = trunk_caches(H, W, C);
   if (cache != nullptr) {
@@ -747,7 +775,7 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
     if (entry != nullptr && continue_chunk) c.cache = entry;
     wvae_status r = conv(c);
     if (r != WVAE_OK || entry == nullptr) return r;
-    return cuda_status(cudaMemcpyAsync(entry, static_cast<const char*>(c.x) + (T - 2) * frame,
+    return cuda_status(cudaMemcpyAsync(entry, static_cast<const char*>(c.x) + (c.T - 2) * frame,
                                        2 * frame, cudaMemcpyDeviceToDevice, s));
   };
   char* ws = static_cast<char*>(workspace);
@@ -792,6 +820,7 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
   }
   for (int stg = 0; stg < 4; ++stg) {
     const int Cs = C[stg];
+    const int Ts = F[stg];
     const size_t frame = static_cast<size_t>(Hs) * Ws * Cs * 2;  // bf16 activation frame
     for (int blk = 0; blk < 2; ++blk) {
       // conv1: A1 -> A2 (norm2 in the epilogue)
@@ -800,7 +829,7 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
       c1.cin_pad = Cs;
       c1.packed = packed[pi++];
       c1.cout = Cs;
-      c1.T = T; c1.H = Hs; c1.W = Ws;
+      c1.T = Ts; c1.H = Hs; c1.W = Ws;
       c1.ep.act = act[1];
       next_norm(&c1.ep.gamma, &c1.ep.beta);
       c1.ep.eps = 1e-12f;
@@ -812,7 +841,7 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
       c2.cin_pad = Cs;
       c2.packed = packed[pi++];
       c2.cout = Cs;
-      c2.T = T; c2.H = Hs; c2.W = Ws;
+      c2.T = Ts; c2.H = Hs; c2.W = Ws;
       c2.ep.residual = h;
       c2.ep.residual_f32 = 1;
       const bool last_block = blk == 1;
@@ -842,8 +871,9 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
       cu.cin_pad = Cs;
       cu.packed = packed[pi++];
       cu.cout = C[stg + 1];
-      cu.T = T; cu.H = Hs; cu.W = Ws;
+      cu.T = Ts; cu.H = Hs; cu.W = Ws;
       cu.phases = 4;
+      if (F[stg + 1] != Ts) cu.tdup = first ? 1 : 2;
       Hs *= 2;
       Ws *= 2;
       cu.ep.out = h;
@@ -855,13 +885,48 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
       if (st != WVAE_OK) return st;
     }
   }
-  // head: A_out -> causal conv to 12 channels -> pixel-shuffled video
+  // head: A_out -> causal conv to 12 channels -> pixel-shuffled video.  At 64
+  // or 128 channels the head kernel puts the temporal and column taps in N.
+  if (C[3] <= 128) {
+    char* entry = cache != nullptr ? static_cast<char*>(cache) + K.off[ck] : nullptr;
+    ++ck;
+    HeadParams hp;
+    std::memset(&hp, 0, sizeof(hp));
+    const PackedLayout L = packed_layout(kHeadOut, C[3], 3, 3, 3, WVAE_BF16);
+    if (!encode_act(&hp.tmA, act[0], C[3], Ws, Hs, F[3], kHeadTileCols, kHeadTileRows + 2))
+      return WVAE_ERR_CUDA;
+    if (entry != nullptr && continue_chunk) {
+      if (!encode_act(&hp.tmC, entry, C[3], Ws, Hs, 2, kHeadTileCols, kHeadTileRows + 2))
+        return WVAE_ERR_CUDA;
+      hp.has_cache = 1;
+    }
+    const void* pk = packed[pi++];
+    if (!encode_weights(&hp.tmB, pk, L.taps * C[3], L.cout_pad, 16)) return WVAE_ERR_CUDA;
+    hp.bias = reinterpret_cast<const float*>(static_cast<const char*>(pk) + L.bias_off);
+    hp.video = static_cast<__nv_bfloat16*>(video);
+    hp.T = F[3];
+    hp.H = Hs;
+    hp.W = Ws;
+    hp.cin = C[3];
+    hp.tiles_w = (Ws + kHeadOutCols - 1) / kHeadOutCols;
+    hp.tiles_h = (Hs + kHeadTileRows - 1) / kHeadTileRows;
+    hp.num_tiles = hp.tiles_w * hp.tiles_h;
+    hp.err = d->err;
+    mark(0);
+    st = cuda_status(launch_head_tc(hp, d->num_sms, s));
+    mark(1);
+    ++launch;
+    if (st != WVAE_OK || entry == nullptr) return st;
+    const size_t frame = static_cast<size_t>(Hs) * Ws * C[3] * 2;
+    return cuda_status(cudaMemcpyAsync(entry, reinterpret_cast<const char*>(act[0]) + (F[3] - 2) * frame,
+                                       2 * frame, cudaMemcpyDeviceToDevice, s));
+  }
   TcConv ch;
   ch.x = act[0];
   ch.cin_pad = C[3];
   ch.packed = packed[pi++];
   ch.cout = kHeadOut;
-  ch.T = T; ch.H = Hs; ch.W = Ws;
+  ch.T = F[3]; ch.H = Hs; ch.W = Ws;
   ch.ep.video = static_cast<__nv_bfloat16*>(video);
   return causal_conv(ch, static_cast<size_t>(Hs) * Ws * C[3] * 2);
 }
@@ -874,7 +939,7 @@ wvae_status wvae_decode_trunk(const void* const* packed, const float* const* nor
                               wvae_dtype dtype, void* workspace, size_t ws_bytes,
                               wvae_stream_t stream) {
   return decode_trunk_impl(packed, norms, z, video, T, H, W, widths, dtype, workspace, ws_bytes,
-                           nullptr, 0, nullptr, 0, 0, stream);
+                           nullptr, 0, nullptr, 0, 0, 0, stream);
 }
 
 wvae_status wvae_decode_trunk_chunk(const void* const* packed, const float* const* norms,
@@ -884,7 +949,16 @@ wvae_status wvae_decode_trunk_chunk(const void* const* packed, const float* cons
                                     int continue_chunk, wvae_stream_t stream) {
   if (cache == nullptr) return WVAE_ERR_INVALID_ARG;
   return decode_trunk_impl(packed, norms, z, video, T, H, W, widths, dtype, workspace, ws_bytes,
-                           nullptr, 0, cache, cache_bytes, continue_chunk, stream);
+                           nullptr, 0, cache, cache_bytes, continue_chunk, 0, stream);
+}
+
+wvae_status wvae_decode_video(const void* const* packed, const float* const* norms, const void* z,
+                              void* video, int T, int H, int W, const int* widths,
+                              wvae_dtype dtype, void* workspace, size_t ws_bytes, void* cache,
+                              size_t cache_bytes, int continue_chunk, wvae_stream_t stream) {
+  if (cache == nullptr && continue_chunk) return WVAE_ERR_INVALID_ARG;
+  return decode_trunk_impl(packed, norms, z, video, T, H, W, widths, dtype, workspace, ws_bytes,
+                           nullptr, 0, cache, cache_bytes, continue_chunk, 1, stream);
 }
 
 wvae_status wvae_decode_trunk_timed(const void* const* packed, const float* const* norms,
@@ -894,7 +968,7 @@ wvae_status wvae_decode_trunk_timed(const void* const* packed, const float* cons
                                     wvae_stream_t stream) {
   if (events == nullptr) return WVAE_ERR_INVALID_ARG;
   return decode_trunk_impl(packed, norms, z, video, T, H, W, widths, dtype, workspace, ws_bytes,
-                           events, n_events, nullptr, 0, 0, stream);
+                           events, n_events, nullptr, 0, 0, 0, stream);
 }
 
 // ------------------------------------------------- res block, no allocation

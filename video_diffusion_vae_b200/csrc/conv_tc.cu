@@ -592,10 +592,13 @@ __device__ __forceinline__ void tmem_store_chunk(uint32_t taddr, const float (&v
 // layer's norm is fused: h = acc + bias (+ residual) goes out raw (if asked),
 // back into the lane (so the second pass reads neither the residual nor the
 // bias again), and into the returned sum of squares.
+// No second output voxel (see the temporal 2x copies in epilogue()).
+constexpr size_t kNoVox = ~static_cast<size_t>(0);
+
 template <int NC>
 __device__ __forceinline__ void pass1_chunk(const ConvParams& p, const Smem& s, uint32_t taddr,
-                                            int c0, int n0, bool valid, size_t vox, float& ss,
-                                            bool keep) {
+                                            int c0, int n0, bool valid, size_t vox, size_t vox2,
+                                            float& ss, bool keep) {
   float v[NC];
   result_chunk<NC>(p, s, taddr, c0, n0, valid, vox, v);
   float2 sa = make_float2(0.0f, 0.0f), sb = sa;  // two packed chains
@@ -606,18 +609,21 @@ __device__ __forceinline__ void pass1_chunk(const ConvParams& p, const Smem& s, 
     sb = ffma2(x1, x1, sb);
   }
   ss += (sa.x + sa.y) + (sb.x + sb.y);
-  if (valid) store_raw<NC>(p, c0, n0, vox, v);
+  if (valid) {
+    store_raw<NC>(p, c0, n0, vox, v);
+    if (vox2 != kNoVox) store_raw<NC>(p, c0, n0, vox2, v);
+  }
   if (keep) tmem_store_chunk<NC>(taddr + c0, v);
 }
 // keep = false: h is not stored back (the caller re-reads it from the fp32
 // raw output instead).
 __device__ __forceinline__ float lane_pass1(const ConvParams& p, const Smem& s, uint32_t taddr,
                                            int c_lo, int c_hi, int n0, bool valid, size_t vox,
-                                           bool keep) {
+                                           size_t vox2, bool keep) {
   float ss = 0.0f;
   int c0 = c_lo;
-  for (; c0 + 32 <= c_hi; c0 += 32) pass1_chunk<32>(p, s, taddr, c0, n0, valid, vox, ss, keep);
-  if (c0 < c_hi) pass1_chunk<16>(p, s, taddr, c0, n0, valid, vox, ss, keep);
+  for (; c0 + 32 <= c_hi; c0 += 32) pass1_chunk<32>(p, s, taddr, c0, n0, valid, vox, vox2, ss, keep);
+  if (c0 < c_hi) pass1_chunk<16>(p, s, taddr, c0, n0, valid, vox, vox2, ss, keep);
   if (keep) tmem_wait_st();
   return ss;
 }
@@ -625,7 +631,7 @@ __device__ __forceinline__ float lane_pass1(const ConvParams& p, const Smem& s, 
 // Second pass reading h back from the fp32 raw output this thread wrote in
 // pass 1 (the accumulator is released already).
 __device__ __forceinline__ void lane_pass2_global(const ConvParams& p, const Smem& s, int n0,
-                                                 bool valid, size_t vox, float rs) {
+                                                 bool valid, size_t vox, size_t vox2, float rs) {
   if (!valid) return;
   const float* h = static_cast<const float*>(p.ep.out) + vox * p.cout + n0;
   int c0 = 0;
@@ -651,6 +657,7 @@ __device__ __forceinline__ void lane_pass2_global(const ConvParams& p, const Sme
       }
     }
     store_act<32>(p, s, c0, n0, vox, rs, v);
+    if (vox2 != kNoVox) store_act<32>(p, s, c0, n0, vox2, rs, v);
   }
   if (c0 < p.BN) {
     float v[16];
@@ -664,40 +671,53 @@ __device__ __forceinline__ void lane_pass2_global(const ConvParams& p, const Sme
       v[4 * q + 3] = f.w;
     }
     store_act<16>(p, s, c0, n0, vox, rs, v);
+    if (vox2 != kNoVox) store_act<16>(p, s, c0, n0, vox2, rs, v);
   }
 }
 
 // Second pass: the next layer's activation SiLU(h r gamma + beta) from h in the lane.
 __device__ __forceinline__ void lane_pass2(const ConvParams& p, const Smem& s, uint32_t taddr,
                                           int c_lo, int c_hi, int n0, bool valid, size_t vox,
-                                          float rs) {
+                                          size_t vox2, float rs) {
   int c0 = c_lo;
   for (; c0 + 32 <= c_hi; c0 += 32) {
     float v[32];
     tmem_load_chunk<32>(taddr + c0, v);
-    if (valid) store_act<32>(p, s, c0, n0, vox, rs, v);
+    if (valid) {
+      store_act<32>(p, s, c0, n0, vox, rs, v);
+      if (vox2 != kNoVox) store_act<32>(p, s, c0, n0, vox2, rs, v);
+    }
   }
   if (c0 < c_hi) {
     float v[16];
     tmem_load_chunk<16>(taddr + c0, v);
-    if (valid) store_act<16>(p, s, c0, n0, vox, rs, v);
+    if (valid) {
+      store_act<16>(p, s, c0, n0, vox, rs, v);
+      if (vox2 != kNoVox) store_act<16>(p, s, c0, n0, vox2, rs, v);
+    }
   }
 }
 
 // Single pass when no norm is fused: raw result and / or video.
 __device__ __forceinline__ void lane_emit(const ConvParams& p, const Smem& s, uint32_t taddr,
                                           int c_lo, int c_hi, int n0, bool valid, size_t vox,
-                                          const TileCoord& tc, int h, int w) {
+                                          size_t vox2, const TileCoord& tc, int h, int w) {
   int c0 = c_lo;
   for (; c0 + 32 <= c_hi; c0 += 32) {
     float v[32];
     result_chunk<32>(p, s, taddr, c0, n0, valid, vox, v);
-    if (valid) emit_chunk<32>(p, c0, n0, tc, h, w, vox, v);
+    if (valid) {
+      emit_chunk<32>(p, c0, n0, tc, h, w, vox, v);
+      if (vox2 != kNoVox) store_raw<32>(p, c0, n0, vox2, v);
+    }
   }
   if (c0 < c_hi) {
     float v[16];
     result_chunk<16>(p, s, taddr, c0, n0, valid, vox, v);
-    if (valid) emit_chunk<16>(p, c0, n0, tc, h, w, vox, v);
+    if (valid) {
+      emit_chunk<16>(p, c0, n0, tc, h, w, vox, v);
+      if (vox2 != kNoVox) store_raw<16>(p, c0, n0, vox2, v);
+    }
   }
 }
 
@@ -755,20 +775,34 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
       const int h = tc.th * p.tile_rows + idx / p.tile_cols;
       const int w = tc.tw * p.out_cols + c - (p.nw > 1 ? 1 : 0);
       const bool valid = h < p.H && w < p.W && (p.nw == 1 || (c >= 1 && c <= p.tile_cols - 2));
-      // output voxel: (t, h, w), or (t, 2h + p', 2w + q') of the 2H x 2W output in phase mode
-      const size_t vox = p.phases == 4
-                             ? (static_cast<size_t>(tc.t) * 2 * p.H + 2 * h + (tc.phase >> 1)) *
+      // output voxel: (t, h, w), or (t, 2h + p', 2w + q') of the 2H x 2W output in phase
+      // mode.  With a temporal 2x step (phase mode only) input frame t goes to output
+      // frames 2t - 1 and 2t (tdup 1: frame 0 of the decode once), or 2t and 2t + 1
+      // (tdup 2: a continuing chunk).
+      int t0 = tc.t, t1 = -1;
+      if (p.tdup == 1) {
+        t0 = tc.t == 0 ? 0 : 2 * tc.t - 1;
+        t1 = tc.t == 0 ? -1 : 2 * tc.t;
+      } else if (p.tdup == 2) {
+        t0 = 2 * tc.t;
+        t1 = 2 * tc.t + 1;
+      }
+      auto out_vox = [&](int to) {
+        return p.phases == 4 ? (static_cast<size_t>(to) * 2 * p.H + 2 * h + (tc.phase >> 1)) *
                                        (2 * p.W) + 2 * w + (tc.phase & 1)
-                             : (static_cast<size_t>(tc.t) * p.H + h) * p.W + w;
+                             : (static_cast<size_t>(to) * p.H + h) * p.W + w;
+      };
+      const size_t vox = out_vox(t0);
+      const size_t vox2 = t1 < 0 ? kNoVox : out_vox(t1);
       const uint32_t n_stride = conv_tc_acc_stride(p);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              (acc * static_cast<uint32_t>(p.S) + static_cast<uint32_t>(sub)) * n_stride;
       if (p.nw > 1) {
         lane_emit_taps_in_n<16>(p, s, taddr, n0, valid, vox, tc, h, w);  // BN = 16
       } else if (p.ep.act == nullptr) {
-        lane_emit(p, s, taddr, 0, p.BN, n0, valid, vox, tc, h, w);
+        lane_emit(p, s, taddr, 0, p.BN, n0, valid, vox, vox2, tc, h, w);
       } else {
-        float ss = lane_pass1(p, s, taddr, 0, p.BN, n0, valid, vox, !early);
+        float ss = lane_pass1(p, s, taddr, 0, p.BN, n0, valid, vox, vox2, !early);
         if (early) {
           tc_fence_before();
           mbar_arrive(smem_u32(&s.tempty[acc]));
@@ -792,9 +826,9 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
         }
         const float rs = rootC / fmaxf(sqrtf(ss), p.ep.eps);
         if (early)
-          lane_pass2_global(p, s, n0, valid, vox, rs);
+          lane_pass2_global(p, s, n0, valid, vox, vox2, rs);
         else
-          lane_pass2(p, s, taddr, 0, p.BN, n0, valid, vox, rs);
+          lane_pass2(p, s, taddr, 0, p.BN, n0, valid, vox, vox2, rs);
       }
     }
     if (!early) {

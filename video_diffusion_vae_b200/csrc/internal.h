@@ -50,6 +50,8 @@ struct ConvParams {
   int cout, cout_pad;
   int KT, KH, KW;
   int phases;        // 4: upsample-conv phase mode (KH = KW = 2, output at (2h+p, 2w+q))
+  int tdup;          // phase mode: a temporal 2x step in the output frames (1: input frame
+                     //    t -> 2t - 1 and 2t, frame 0 once; 2: t -> 2t and 2t + 1)
   int nsplit;        // 2: a cluster of 2 CTAs splits N (rank = N tile) and exchanges the
                      //    RMS partial sums over distributed shared memory
   int has_cache;
@@ -135,6 +137,29 @@ cudaError_t launch_upsample2x(const void* x, void* y, int elem_bytes, int T, int
                               cudaStream_t stream);
 // fp32 [n] -> bf16 [n]
 cudaError_t launch_f32_to_bf16(const float* x, __nv_bfloat16* y, size_t n, cudaStream_t stream);
+
+// ------------------------------------------------------------- head (tcgen05)
+// The decoder head (causal 3x3x3 conv C -> 12, 2x2 pixel shuffle into the
+// NCDHW video) with the 3 temporal x 3 column taps in N (N = 144); see
+// head_tc.cu.  C = 64 or 128.
+constexpr int kHeadTileRows = 8;
+constexpr int kHeadTileCols = 16;   // computed columns; 14 are output
+constexpr int kHeadOutCols = 14;
+constexpr int kHeadThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+
+struct HeadParams {
+  CUtensorMap tmA;   // activation bf16 [T][H][W][cin], box {64, 16, 10, 1}
+  CUtensorMap tmC;   // cached frames bf16 [2][H][W][cin], same box (has_cache)
+  CUtensorMap tmB;   // packed weights bf16 [16][27 * cin] (standard prepack), box {64, 16}
+  const float* bias; // fp32 [16] (packed blob)
+  __nv_bfloat16* video;  // [3][T][2H][2W]
+  int T, H, W, cin;
+  int tiles_w, tiles_h, num_tiles;
+  int has_cache;     // frames -2, -1 come from tmC
+  unsigned* err;
+};
+size_t head_tc_smem_bytes(int cin);
+cudaError_t launch_head_tc(const HeadParams& p, int num_sms, cudaStream_t stream);
 
 // Device error word (defined in api.cu).
 unsigned* device_error_word();

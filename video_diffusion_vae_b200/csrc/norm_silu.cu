@@ -133,13 +133,14 @@ __global__ void __launch_bounds__(kNormThreads, (VEC == 8 && CH <= 4) ? 3 : 2) n
 }
 
 // ------------------------------------------------------- bf16: TMA-fed ring
-constexpr int kRingWarps = 16;                       // consumer warps
-constexpr int kRingThreads = 32 * (1 + kRingWarps);  // + the copy warp
 constexpr int kRingStages = 3;
 constexpr int kRingChunkBytes = 65536;
 
-template <int CH>
-__global__ void __launch_bounds__(kRingThreads, 1)
+// CH: 16-byte vectors per lane; V: voxels a lane group carries through one
+// pass (their load, reduction and output chains interleave, hiding the
+// latency of each); NW: consumer warps.
+template <int CH, int V, int NW>
+__global__ void __launch_bounds__(32 * (NW + 1), 1)
     norm_silu_ring_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* y,
                           const float* __restrict__ gamma, const float* __restrict__ beta,
                           long nvox, int C, int L, int vpc, float eps, unsigned* err) {
@@ -152,7 +153,7 @@ __global__ void __launch_bounds__(kRingThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kRingStages; ++i) {
       mbar_init(smem_u32(&full[i]), 1);
-      mbar_init(smem_u32(&empty[i]), kRingWarps);
+      mbar_init(smem_u32(&empty[i]), NW);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -219,44 +220,58 @@ __global__ void __launch_bounds__(kRingThreads, 1)
     const long v0 = ch * vpc;
     const int nv = nvox - v0 < vpc ? static_cast<int>(nvox - v0) : vpc;
     const uint8_t* stage = smem_raw + st * chunk_bytes;
-    // warp-uniform bound: the shuffles need every lane
-    for (int vb = cw * gpw; vb < nv; vb += kRingWarps * gpw) {
-      const int vl = vb + grp;
-      const bool live = vl < nv;
-      const uint4* src = reinterpret_cast<const uint4*>(stage + static_cast<size_t>(vl) * C * 2);
-      // the lane's channel pairs, unpacked once for both passes
-      float2 xp[CH][4];
-      float2 ssa = make_float2(0.0f, 0.0f), ssb = ssa;  // two packed chains
+    // A warp takes gpw * V consecutive voxels per pass: lane group grp holds
+    // voxels vb + grp + j gpw, j < V.  The bound is warp-uniform (the shuffles
+    // need every lane).
+    for (int vb = cw * gpw * V; vb < nv; vb += NW * gpw * V) {
+      float2 xp[V][CH][4];
+      float ss[V];
 #pragma unroll
-      for (int k = 0; k < CH; ++k) {
-        const int vi = sub + k * L;
-        const uint4 raw = (live && vi < nvec) ? src[vi] : make_uint4(0u, 0u, 0u, 0u);
-        xp[k][0] = make_float2(bf16lo(raw.x), bf16hi(raw.x));
-        xp[k][1] = make_float2(bf16lo(raw.y), bf16hi(raw.y));
-        xp[k][2] = make_float2(bf16lo(raw.z), bf16hi(raw.z));
-        xp[k][3] = make_float2(bf16lo(raw.w), bf16hi(raw.w));
-        ssa = ffma2(xp[k][0], xp[k][0], ssa);
-        ssb = ffma2(xp[k][1], xp[k][1], ssb);
-        ssa = ffma2(xp[k][2], xp[k][2], ssa);
-        ssb = ffma2(xp[k][3], xp[k][3], ssb);
-      }
-      float ss = (ssa.x + ssa.y) + (ssb.x + ssb.y);
-      for (int off = L >> 1; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-      // sqrt(C) / max(||x||, eps) = sqrt(C) * rsqrt(max(ss, eps^2)) while eps^2 is normal
-      const float r = eps2_normal ? rootC * rsqrtf(fmaxf(ss, eps2)) : rootC / fmaxf(sqrtf(ss), eps);
-      const float2 r2 = make_float2(r, r);
-      uint4* dst = reinterpret_cast<uint4*>(y + (v0 + vl) * C);
+      for (int j = 0; j < V; ++j) {
+        const int vl = vb + grp + j * gpw;
+        const bool live = vl < nv;
+        const uint4* src = reinterpret_cast<const uint4*>(stage + static_cast<size_t>(vl) * C * 2);
+        float2 ssa = make_float2(0.0f, 0.0f), ssb = ssa;  // two packed chains
 #pragma unroll
-      for (int k = 0; k < CH; ++k) {
-        const int vi = sub + k * L;
-        if (!live || vi >= nvec) continue;
-        uint32_t w4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 o = silu_half2(ffma2(xp[k][e], fmul2(r2, g[k][e]), b[k][e]));
-          w4[e] = pack_bf16x2(o.x, o.y);
+        for (int k = 0; k < CH; ++k) {
+          const int vi = sub + k * L;
+          const uint4 raw = (live && vi < nvec) ? src[vi] : make_uint4(0u, 0u, 0u, 0u);
+          xp[j][k][0] = make_float2(bf16lo(raw.x), bf16hi(raw.x));
+          xp[j][k][1] = make_float2(bf16lo(raw.y), bf16hi(raw.y));
+          xp[j][k][2] = make_float2(bf16lo(raw.z), bf16hi(raw.z));
+          xp[j][k][3] = make_float2(bf16lo(raw.w), bf16hi(raw.w));
+          ssa = ffma2(xp[j][k][0], xp[j][k][0], ssa);
+          ssb = ffma2(xp[j][k][1], xp[j][k][1], ssb);
+          ssa = ffma2(xp[j][k][2], xp[j][k][2], ssa);
+          ssb = ffma2(xp[j][k][3], xp[j][k][3], ssb);
         }
-        dst[vi] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        ss[j] = (ssa.x + ssa.y) + (ssb.x + ssb.y);
+      }
+      for (int off = L >> 1; off > 0; off >>= 1) {
+#pragma unroll
+        for (int j = 0; j < V; ++j) ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], off);
+      }
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        const int vl = vb + grp + j * gpw;
+        const bool live = vl < nv;
+        // sqrt(C) / max(||x||, eps) = sqrt(C) * rsqrt(max(ss, eps^2)) while eps^2 is normal
+        const float r = eps2_normal ? rootC * rsqrtf(fmaxf(ss[j], eps2))
+                                    : rootC / fmaxf(sqrtf(ss[j]), eps);
+        const float2 r2 = make_float2(r, r);
+        uint4* dst = reinterpret_cast<uint4*>(y + (v0 + vl) * C);
+#pragma unroll
+        for (int k = 0; k < CH; ++k) {
+          const int vi = sub + k * L;
+          if (!live || vi >= nvec) continue;
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 o = silu_half2(ffma2(xp[j][k][e], fmul2(r2, g[k][e]), b[k][e]));
+            w4[e] = pack_bf16x2(o.x, o.y);
+          }
+          dst[vi] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
       }
     }
     __syncwarp();
@@ -264,21 +279,21 @@ __global__ void __launch_bounds__(kRingThreads, 1)
   }
 }
 
-template <int CH>
+template <int CH, int V, int NW>
 cudaError_t launch_ring(const __nv_bfloat16* x, __nv_bfloat16* y, const float* gamma,
                         const float* beta, long nvox, int C, int L, float eps, int num_sms,
                         cudaStream_t stream) {
   int vpc = kRingChunkBytes / (C * 2);
   if (vpc < 1) vpc = 1;
   const size_t smem = static_cast<size_t>(kRingStages) * vpc * C * 2 + 2 * kRingStages * 8 + 16;
-  auto kern = norm_silu_ring_kernel<CH>;
+  auto kern = norm_silu_ring_kernel<CH, V, NW>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const long nchunks = (nvox + vpc - 1) / vpc;
   const int grid = nchunks < num_sms ? static_cast<int>(nchunks) : num_sms;
-  kern<<<grid, kRingThreads, smem, stream>>>(x, y, gamma, beta, nvox, C, L, vpc, eps,
-                                             device_error_word());
+  kern<<<grid, 32 * (NW + 1), smem, stream>>>(x, y, gamma, beta, nvox, C, L, vpc, eps,
+                                              device_error_word());
   return cudaGetLastError();
 }
 
@@ -324,9 +339,9 @@ cudaError_t launch_norm_silu_bf16(const __nv_bfloat16* x, __nv_bfloat16* y, cons
   int L = 1;
   while (L < nvec && L < 32) L <<= 1;
   const int ch = (nvec + L - 1) / L;
-  if (ch == 1) return launch_ring<1>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
-  if (ch == 2) return launch_ring<2>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
-  if (ch <= 4) return launch_ring<4>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
+  if (ch == 1) return launch_ring<1, 2, 16>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
+  if (ch == 2) return launch_ring<2, 2, 16>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
+  if (ch <= 4) return launch_ring<4, 1, 16>(x, y, gamma, beta, nvox, C, L, eps, num_sms, stream);
   return cudaErrorInvalidValue;
 }
 
