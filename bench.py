@@ -400,7 +400,31 @@ def components(peaks, flush, reps=10):
     out["conv_512x512_4x88x156"] = {"ms": med, "TFLOP/s": fl / med / 1e9,
                                     "frac_bf16": fl / med / 1e9 / peaks["bf16_tflops"],
                                     "frac_2250": fl / med / 1e9 / 2250.0}
-    del xd, y, pk
+    # the same conv as Winograd F(2x2, 3x3) products (same box, same flush)
+    pw = B.prepack_conv_winograd(w.cuda().bfloat16(), b.cuda())
+    wsw = torch.empty(B.load().wvae_causal_conv3d_winograd_workspace_bytes(4, 88, 156, 512, 512),
+                      dtype=torch.uint8, device="cuda")
+    med, mn = time_events(lambda: B.causal_conv3d_winograd(xd, pw, out=y, workspace=wsw), reps, 3, flush)
+    out["conv_512x512_4x88x156_winograd"] = {
+        "ms": med, "TFLOP/s_dense_equiv": fl / med / 1e9,
+        "frac_bf16_dense_equiv": fl / med / 1e9 / peaks["bf16_tflops"],
+        "vs_direct": out["conv_512x512_4x88x156"]["ms"] / med}
+    del xd, y, pk, pw, wsw
+    # a 256-channel layer of the trunk's stage 2, direct and Winograd
+    x, w, b = synth.conv_input(cin=256, cout=256, T=4, H=176, W=312, seed=0)
+    xd = x.permute(1, 2, 3, 0).contiguous().cuda().bfloat16()
+    y = torch.empty_like(xd)
+    pk = B.prepack_conv(w.cuda().bfloat16(), b.cuda())
+    pw = B.prepack_conv_winograd(w.cuda().bfloat16(), b.cuda())
+    wsw = torch.empty(B.load().wvae_causal_conv3d_winograd_workspace_bytes(4, 176, 312, 256, 256),
+                      dtype=torch.uint8, device="cuda")
+    fl = 2.0 * 256 * 256 * 27 * 4 * 176 * 312
+    md, _ = time_events(lambda: B.causal_conv3d(xd, pk, out=y), reps, 3, flush)
+    mw, _ = time_events(lambda: B.causal_conv3d_winograd(xd, pw, out=y, workspace=wsw), reps, 3, flush)
+    out["conv_256x256_4x176x312"] = {"ms": md, "TFLOP/s": fl / md / 1e9}
+    out["conv_256x256_4x176x312_winograd"] = {"ms": mw, "TFLOP/s_dense_equiv": fl / mw / 1e9,
+                                               "vs_direct": md / mw}
+    del xd, y, pk, pw, wsw
     for cout in (256, 128):
         x, p = synth.resblock_input(cout=cout)
         blk = B.PackedResBlock(p)

@@ -145,6 +145,37 @@ WVAE_API wvae_status wvae_causal_conv3d(const void* x, const void* cache, const 
                                const void* residual, void* y, wvae_dtype dtype, void* workspace,
                                size_t ws_bytes, wvae_stream_t stream);
 
+/* ------------------------------------------- causal conv3d, Winograd form
+ * The same causal 3x3x3 conv as wvae_causal_conv3d (bf16, no norm, no cache),
+ * computed as Winograd F(2x2, 3x3) products (Lavin and Gray's minimal
+ * filtering) the way the page-3 decoder computes its convs (FastVideo
+ * README, "Use": Winograd transforms of the weights; "Performance and
+ * memory": the products take 60 % of its GPU time).  Spatially Winograd,
+ * temporally direct: the 16 transform planes of the input, V = B^T d B per
+ * 4 x 4 tile at stride 2, are multiplied on the tensor cores by the
+ * transformed weights U = G g G^T of each temporal tap (fp16 operands, fp32
+ * accumulation) and the products go through Y = A^T M A, + bias (+ residual).
+ * 2.25x fewer tensor-core FLOPs than the direct conv, at the cost of the
+ * planes' memory traffic; fp16 operands keep the direct conv's accuracy.
+ *   packed_w: wvae_conv_winograd_packed_bytes(cout, cin) bytes from
+ *     wvae_prepack_conv_winograd (weights [cout][cin][3][3][3], fp32 or bf16).
+ *   x: [T][H][W][cin] bf16; residual: NULL or [T][H][W][cout] bf16;
+ *   y: [T][H][W][cout] bf16 (no overlap with x or residual).
+ *   workspace: wvae_causal_conv3d_winograd_workspace_bytes(T, H, W, cin, cout)
+ *     bytes: the input planes and the products, fp16
+ *     [16][T][ceil(H/2)][ceil(W/2)][C] each.
+ * cin % 64 == 0, cout % 16 == 0 and cout <= 256 or cout == 512.
+ */
+WVAE_API size_t wvae_conv_winograd_packed_bytes(int cout, int cin);
+WVAE_API wvae_status wvae_prepack_conv_winograd(const void* w, wvae_dtype w_dtype, const float* bias,
+                                                int cout, int cin, void* packed, size_t packed_bytes,
+                                                wvae_stream_t stream);
+WVAE_API size_t wvae_causal_conv3d_winograd_workspace_bytes(int T, int H, int W, int cin, int cout);
+WVAE_API wvae_status wvae_causal_conv3d_winograd(const void* x, const void* packed_w, int T, int H,
+                                                 int W, int cin, int cout, const void* residual,
+                                                 void* y, void* workspace, size_t ws_bytes,
+                                                 wvae_stream_t stream);
+
 /* ------------------------------------------------------------ residual block
  * h = shortcut(x) + conv2(A2(conv1(A1(x)))), A_k = SiLU(norm_k(.)), causal
  * 3x3x3 convs; shortcut = identity when cin == cout, else the 1x1x1 conv

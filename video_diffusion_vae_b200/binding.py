@@ -75,6 +75,10 @@ def load(path: str | None = None):
             "wvae_decode_trunk_cache_bytes": (S, [I, I, ctypes.POINTER(I)]),
             "wvae_decode_trunk_chunk": (I, [ctypes.POINTER(V), ctypes.POINTER(V), V, V, I, I, I,
                                             ctypes.POINTER(I), I, V, S, V, S, I, V]),
+            "wvae_conv_winograd_packed_bytes": (S, [I, I]),
+            "wvae_prepack_conv_winograd": (I, [V, I, V, I, I, V, S, V]),
+            "wvae_causal_conv3d_winograd_workspace_bytes": (S, [I, I, I, I, I]),
+            "wvae_causal_conv3d_winograd": (I, [V, V, I, I, I, I, I, V, V, V, S, V]),
             "wvae_decode_video_frames": (I, [I, I]),
             "wvae_decode_video_workspace_bytes": (S, [I, I, I, ctypes.POINTER(I)]),
             "wvae_decode_video": (I, [ctypes.POINTER(V), ctypes.POINTER(V), V, V, I, I, I,
@@ -248,6 +252,39 @@ def causal_conv3d(x, packed: PackedConv, cache=None, norm=None, residual=None, o
     _check("wvae_causal_conv3d", lib.wvae_causal_conv3d(
         _ptr(x), _ptr(cache), packed.ptr(), T, H, W, cin, cout, kt, kh, kw, _ptr(g), _ptr(b),
         _ptr(residual), _ptr(y), dt, _ptr(ws), nws, _stream()))
+    return y
+
+
+# ------------------------------------------------ causal conv, Winograd form
+def prepack_conv_winograd(w, bias=None) -> PackedConv:
+    """w: PyTorch [Cout, Cin, 3, 3, 3] (fp32 or bf16, CUDA) -> the Winograd-transformed
+    weights (fp16) for causal_conv3d_winograd."""
+    _cuda(w, "w")
+    cout, cin, kt, kh, kw = w.shape
+    if (kt, kh, kw) != (3, 3, 3):
+        raise ValueError("Winograd weights must be [Cout, Cin, 3, 3, 3]")
+    n = load().wvae_conv_winograd_packed_bytes(cout, cin)
+    blob = torch.empty(n, dtype=torch.uint8, device=w.device)
+    b = None if bias is None else _f32vec(bias, cout, "bias")
+    _check("wvae_prepack_conv_winograd", load().wvae_prepack_conv_winograd(
+        _ptr(w), _dt(w), _ptr(b), cout, cin, _ptr(blob), n, _stream()))
+    return PackedConv(blob, cout, cin, (3, 3, 3), BF16)
+
+
+def causal_conv3d_winograd(x, packed: PackedConv, residual=None, out=None, workspace=None):
+    """The causal 3x3x3 conv of x [T, H, W, Cin] bf16 as Winograd F(2x2, 3x3) products."""
+    _cuda(x, "x", torch.bfloat16)
+    T, H, W, cin = x.shape
+    cout = packed.cout
+    y = torch.empty((T, H, W, cout), dtype=x.dtype, device=x.device) if out is None else \
+        _cuda(out, "out", x.dtype, (T, H, W, cout))
+    if residual is not None:
+        _cuda(residual, "residual", x.dtype, (T, H, W, cout))
+    lib = load()
+    ws = _ws(workspace, lib.wvae_causal_conv3d_winograd_workspace_bytes(T, H, W, cin, cout), x.device)
+    _check("wvae_causal_conv3d_winograd", lib.wvae_causal_conv3d_winograd(
+        _ptr(x), packed.ptr(), T, H, W, cin, cout, _ptr(residual), _ptr(y), _ptr(ws), _nbytes(ws),
+        _stream()))
     return y
 
 

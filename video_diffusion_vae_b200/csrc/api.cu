@@ -122,12 +122,30 @@ bool encode_act(CUtensorMap* m, const void* base, int C, int W, int H, int T, in
          CUDA_SUCCESS;
 }
 
-bool encode_weights(CUtensorMap* m, const void* base, int K, int N, int box_rows) {
+// The 16 Winograd transform planes [16][T][H][W][C] fp16 (H x W: the tile grid).
+bool encode_planes(CUtensorMap* m, const void* base, int C, int W, int H, int T, int box_w,
+                   int box_h) {
+  cuuint64_t dims[5] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(W),
+                        static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T), 16};
+  cuuint64_t strides[4] = {static_cast<cuuint64_t>(C) * 2, static_cast<cuuint64_t>(C) * 2 * W,
+                           static_cast<cuuint64_t>(C) * 2 * W * H,
+                           static_cast<cuuint64_t>(C) * 2 * W * H * T};
+  cuuint32_t box[5] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_w),
+                       static_cast<cuuint32_t>(box_h), 1, 1};
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 5, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+bool encode_weights(CUtensorMap* m, const void* base, int K, int N, int box_rows,
+                    CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t es[2] = {1, 1};
-  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+  return g_encode(m, type, 2, const_cast<void*>(base), dims, strides,
                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
@@ -146,6 +164,7 @@ struct TcConv {
   int T = 0, H = 0, W = 0;
   int phases = 1;            // 4: upsample-conv phase mode (packed by prepack_upsample)
   int tdup = 0;              // phase mode: temporal 2x copies of the output (ConvParams::tdup)
+  int wino = 0;              // Winograd products over the 16 transform planes (ConvParams::wino)
   ConvEpilogue ep{};
 };
 
@@ -156,8 +175,14 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
     a.KH = 2;
     a.KW = 2;
   }
-  // phase mode packs 4 phases x 4 taps along K
+  if (a.wino) {  // 16 planes x KT temporal taps, 1 x 1 spatially
+    a.phases = 16;
+    a.KH = 1;
+    a.KW = 1;
+  }
+  // phase mode packs 4 phases x 4 taps along K, Winograd 16 planes x KT taps
   const PackedLayout L = a.phases == 4 ? packed_layout(a.cout, a.cin_pad, 1, 4, 4, WVAE_BF16)
+                         : a.wino      ? packed_layout(a.cout, a.cin_pad, a.KT, 16, 1, WVAE_BF16)
                                        : packed_layout(a.cout, a.cin_pad, a.KT, a.KH, a.KW, WVAE_BF16);
   ConvParams p;
   std::memset(&p, 0, sizeof(p));
@@ -173,6 +198,7 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   p.KW = a.KW;
   p.phases = a.phases;
   p.tdup = a.phases == 4 ? a.tdup : 0;
+  p.wino = a.wino;
   p.has_cache = a.cache != nullptr;
   // The fused norm needs every output channel of a voxel: one CTA holds them
   // all (BN = Cout) up to 256; at 512 a cluster of two CTAs splits N and swaps
@@ -245,10 +271,18 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   p.err = d.err;
   const int box_rows = p.BN;  // BN <= 256
   const int a_rows = static_cast<int>(conv_tc_a_rows(p));
-  if (!encode_act(&p.tmA, a.x, a.cin_pad, a.W, a.H, a.T, p.tile_cols, a_rows))
-    return WVAE_ERR_CUDA;
-  if (!encode_weights(&p.tmB, a.packed, L.taps * a.cin_pad, L.cout_pad, box_rows))
-    return WVAE_ERR_CUDA;
+  if (a.wino) {
+    if (!encode_planes(&p.tmA, a.x, a.cin_pad, a.W, a.H, a.T, p.tile_cols, a_rows))
+      return WVAE_ERR_CUDA;
+    if (!encode_weights(&p.tmB, a.packed, L.taps * a.cin_pad, L.cout_pad, box_rows,
+                        CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+      return WVAE_ERR_CUDA;
+  } else {
+    if (!encode_act(&p.tmA, a.x, a.cin_pad, a.W, a.H, a.T, p.tile_cols, a_rows))
+      return WVAE_ERR_CUDA;
+    if (!encode_weights(&p.tmB, a.packed, L.taps * a.cin_pad, L.cout_pad, box_rows))
+      return WVAE_ERR_CUDA;
+  }
   if (a.cache != nullptr && !encode_act(&p.tmC, a.cache, a.cin_pad, a.W, a.H, a.KT - 1, p.tile_cols,
                                         a_rows))
     return WVAE_ERR_CUDA;
@@ -437,6 +471,90 @@ wvae_status wvae_causal_conv3d(const void* x, const void* cache, const void* pac
   c.ep.out = y;
   c.ep.out_f32 = 0;
   return run_tc_conv(*d, c, s);
+}
+
+// ---------------------------------------------------- Winograd F(2x2, 3x3)
+namespace {
+// Packed Winograd weights: fp16 U [cout_pad][16 x 3][cin_pad], then a zero
+// bias (the products take none) and the conv's bias, fp32 [cout_pad] each.
+PackedLayout wino_layout(int cout, int cin) {
+  PackedLayout L = packed_layout(cout, cin, 3, 16, 1, WVAE_BF16);
+  L.total += static_cast<size_t>(L.cout_pad) * 4;
+  return L;
+}
+size_t wino_planes_bytes(int T, int H, int W, int C) {
+  return round_up_sz(16ull * T * ((H + 1) / 2) * ((W + 1) / 2) * C * 2, 256);
+}
+}  // namespace
+
+size_t wvae_conv_winograd_packed_bytes(int cout, int cin) {
+  if (cout < 1 || cin < 1) return 0;
+  return wino_layout(cout, cin).total;
+}
+
+wvae_status wvae_prepack_conv_winograd(const void* w, wvae_dtype w_dtype, const float* bias,
+                                       int cout, int cin, void* packed, size_t packed_bytes,
+                                       wvae_stream_t stream) {
+  if (!w || !packed) return WVAE_ERR_INVALID_ARG;
+  if (cout < 1 || cin < 1) return WVAE_ERR_INVALID_ARG;
+  if (w_dtype != WVAE_BF16 && w_dtype != WVAE_F32) return WVAE_ERR_UNSUPPORTED;
+  if (!a16(packed)) return WVAE_ERR_ALIGNMENT;
+  const PackedLayout L = wino_layout(cout, cin);
+  if (packed_bytes < L.total) return WVAE_ERR_WORKSPACE;
+  DeviceInfo* d = nullptr;
+  wvae_status st = device_info(&d);
+  if (st != WVAE_OK) return st;
+  float* bias_zero = reinterpret_cast<float*>(static_cast<char*>(packed) + L.bias_off);
+  return cuda_status(launch_wino_prepack(w, w_dtype == WVAE_F32, bias, cout, cin, L.cout_pad,
+                                         L.cin_pad, static_cast<__half*>(packed), bias_zero,
+                                         bias_zero + L.cout_pad,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t wvae_causal_conv3d_winograd_workspace_bytes(int T, int H, int W, int cin, int cout) {
+  if (T < 1 || H < 1 || W < 1 || cin < 1 || cout < 1) return 0;
+  return wino_planes_bytes(T, H, W, cin) + wino_planes_bytes(T, H, W, cout);
+}
+
+wvae_status wvae_causal_conv3d_winograd(const void* x, const void* packed_w, int T, int H, int W,
+                                        int cin, int cout, const void* residual, void* y,
+                                        void* workspace, size_t ws_bytes, wvae_stream_t stream) {
+  if (!x || !packed_w || !y || !workspace) return WVAE_ERR_INVALID_ARG;
+  if (T < 1 || H < 1 || W < 1 || cin < 1 || cout < 1) return WVAE_ERR_INVALID_ARG;
+  if (x == y || (residual != nullptr && residual == y)) return WVAE_ERR_INVALID_ARG;
+  if (!a16(x) || !a16(y) || !a16(packed_w) || !a16(workspace) || (residual && !a16(residual)))
+    return WVAE_ERR_ALIGNMENT;
+  if (cin % 64 != 0 || !bf16_cout_ok(cout)) return WVAE_ERR_UNSUPPORTED;
+  if (ws_bytes < wvae_causal_conv3d_winograd_workspace_bytes(T, H, W, cin, cout))
+    return WVAE_ERR_WORKSPACE;
+  DeviceInfo* d = nullptr;
+  wvae_status st = device_info(&d);
+  if (st != WVAE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  __half* v = static_cast<__half*>(workspace);
+  __half* m = reinterpret_cast<__half*>(static_cast<char*>(workspace) +
+                                        wino_planes_bytes(T, H, W, cin));
+  st = cuda_status(launch_wino_input(static_cast<const __nv_bfloat16*>(x), v, T, H, W, cin, s));
+  if (st != WVAE_OK) return st;
+  TcConv c;
+  c.x = v;
+  c.cin_pad = cin;
+  c.packed = packed_w;
+  c.cout = cout;
+  c.KT = 3;
+  c.T = T;
+  c.H = (H + 1) / 2;
+  c.W = (W + 1) / 2;
+  c.wino = 1;
+  c.ep.out = m;
+  c.ep.out_f16 = 1;
+  st = run_tc_conv(*d, c, s);
+  if (st != WVAE_OK) return st;
+  const PackedLayout L = wino_layout(cout, cin);
+  const float* bias = reinterpret_cast<const float*>(static_cast<const char*>(packed_w) + L.bias_off) +
+                      L.cout_pad;
+  return cuda_status(launch_wino_output(m, bias, static_cast<const __nv_bfloat16*>(residual),
+                                        static_cast<__nv_bfloat16*>(y), T, H, W, cout, s));
 }
 
 // ------------------------------------------------------------ residual block

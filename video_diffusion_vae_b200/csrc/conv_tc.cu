@@ -170,7 +170,8 @@ __device__ void producer(const ConvParams& p, const Smem& s, int crank) {
     // mode: output (2h+p', 2w+q') reads rows h + p' - 1 + r, columns w + q' - 1 + c
     const int oh = p.phases == 4 ? (tc.phase >> 1) - 1 : -(p.KH - 1) / 2;
     const int ow = p.phases == 4 ? (tc.phase & 1) - 1 : -(p.KW - 1) / 2;
-    const int tap0 = p.phases == 4 ? tc.phase * 4 : 0;
+    // phase mode: phase p's 4 taps; Winograd: transform plane xi's KT temporal taps
+    const int tap0 = p.phases == 4 ? tc.phase * 4 : (p.wino ? tc.phase * p.KT : 0);
     for (int g = 0; g < p.groups; ++g) {
       const bool main_seg = g < p.groups_main;
       int kt = 0, kw = 0, cc;
@@ -187,7 +188,9 @@ __device__ void producer(const ConvParams& p, const Smem& s, int crank) {
       auto load_a = [&](uint32_t dst, uint32_t bar) {
         if (main_seg) {
           const int ts = tc.t + kt - (p.KT - 1);
-          if (ts < 0 && p.has_cache)
+          if (p.wino)
+            tma_load_5d(dst, &p.tmA, bar, cc * kBK, w0, h0, ts, tc.phase);
+          else if (ts < 0 && p.has_cache)
             tma_load_4d(dst, &p.tmC, bar, cc * kBK, w0 + ow + kw, h0 + oh, ts + p.KT - 1);
           else
             tma_load_4d(dst, &p.tmA, bar, cc * kBK, w0 + ow + kw, h0 + oh, ts);
@@ -269,7 +272,8 @@ __device__ void mma_issuer(const ConvParams& p, const Smem& s, uint32_t tmem_bas
   static_assert(BT == 1 || BT == KHT, "a B stage holds one weight tile or the group's row taps");
   static_assert(!COMBINED || BT == KHT, "a combined stage holds all of a group's weight tiles");
   const uint32_t n_mma = static_cast<uint32_t>(p.nw * p.BN);  // N of one MMA
-  const uint32_t idesc = umma_idesc_bf16(kBM, static_cast<int>(n_mma));
+  const uint32_t idesc = p.wino ? umma_idesc_f16(kBM, static_cast<int>(n_mma))
+                                : umma_idesc_bf16(kBM, static_cast<int>(n_mma));
   // Descriptors of stage 0 of each ring; the start field counts 16-byte units.
   const uint64_t adesc0 = umma_desc_sw128(smem_u32(s.a_ring));
   const uint64_t bdesc0 = umma_desc_sw128(smem_u32(s.b_ring));
@@ -461,6 +465,15 @@ __device__ __forceinline__ void store_bf16(__nv_bfloat16* dst, const float (&v)[
 }
 
 template <int NC>
+__device__ __forceinline__ void store_f16(__half* dst, const float (&v)[NC]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < NC / 8; ++q)
+    d[q] = make_uint4(pack_f16x2(v[8 * q], v[8 * q + 1]), pack_f16x2(v[8 * q + 2], v[8 * q + 3]),
+                      pack_f16x2(v[8 * q + 4], v[8 * q + 5]), pack_f16x2(v[8 * q + 6], v[8 * q + 7]));
+}
+
+template <int NC>
 __device__ __forceinline__ void store_f32(float* dst, const float (&v)[NC], bool vec32) {
   if (vec32) {
 #pragma unroll
@@ -504,6 +517,8 @@ __device__ __forceinline__ void store_raw(const ConvParams& p, int c0, int n0, s
     const size_t off = ovox * p.cout + n0 + c0;
     if (ep.out_f32)
       store_f32<NC>(static_cast<float*>(ep.out) + off, v, ep.vec32 != 0);
+    else if (ep.out_f16)
+      store_f16<NC>(static_cast<__half*>(ep.out) + off, v);
     else
       store_bf16<NC>(static_cast<__nv_bfloat16*>(ep.out) + off, v, ep.vec32 != 0);
   }
@@ -788,6 +803,8 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
         t1 = 2 * tc.t + 1;
       }
       auto out_vox = [&](int to) {
+        if (p.wino)  // transform plane xi = phase of the products
+          return ((static_cast<size_t>(tc.phase) * p.T + to) * p.H + h) * p.W + w;
         return p.phases == 4 ? (static_cast<size_t>(to) * 2 * p.H + 2 * h + (tc.phase >> 1)) *
                                        (2 * p.W) + 2 * w + (tc.phase & 1)
                              : (static_cast<size_t>(to) * p.H + h) * p.W + w;

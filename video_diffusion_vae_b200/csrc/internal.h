@@ -2,6 +2,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstddef>
@@ -28,7 +29,8 @@ struct ConvEpilogue {
   const void* residual;     // [T][H][W][cout] or null
   int residual_f32;         // residual dtype: 1 fp32, 0 bf16
   void* out;                // raw result [T][H][W][cout] ([T][2H][2W][cout] in phase mode), or null
-  int out_f32;              // out dtype: 1 fp32, 0 bf16
+  int out_f32;              // out dtype: 1 fp32, 0 bf16 (or fp16 with out_f16)
+  int out_f16;              // out is fp16 (the Winograd products)
   __nv_bfloat16* act;       // SiLU(norm(result)) bf16 [T][H][W][cout], or null
   const float* gamma;       // fp32 [cout] for act
   const float* beta;        // fp32 [cout] for act
@@ -50,6 +52,9 @@ struct ConvParams {
   int cout, cout_pad;
   int KT, KH, KW;
   int phases;        // 4: upsample-conv phase mode (KH = KW = 2, output at (2h+p, 2w+q))
+  int wino;          // 1: Winograd products: phases = 16 transform planes, fp16 operands, A
+                     //    = the planes [16][T][H][W][cin] (tmA 5-D, H x W = the tile grid),
+                     //    weights [cout_pad][16 x KT][cin_pad], out [16][T][H][W][cout]
   int tdup;          // phase mode: a temporal 2x step in the output frames (1: input frame
                      //    t -> 2t - 1 and 2t, frame 0 once; 2: t -> 2t and 2t + 1)
   int nsplit;        // 2: a cluster of 2 CTAs splits N (rank = N tile) and exchanges the
@@ -160,6 +165,15 @@ struct HeadParams {
 };
 size_t head_tc_smem_bytes(int cin);
 cudaError_t launch_head_tc(const HeadParams& p, int num_sms, cudaStream_t stream);
+
+// ---------------------------------------------------- Winograd F(2x2, 3x3)
+cudaError_t launch_wino_prepack(const void* w, bool is_f32, const float* bias, int cout, int cin,
+                                int cout_pad, int cin_pad, __half* up, float* bias_zero,
+                                float* bias_p, cudaStream_t stream);
+cudaError_t launch_wino_input(const __nv_bfloat16* x, __half* v, int T, int H, int W, int C,
+                              cudaStream_t stream);
+cudaError_t launch_wino_output(const __half* m, const float* bias, const __nv_bfloat16* residual,
+                               __nv_bfloat16* y, int T, int H, int W, int C, cudaStream_t stream);
 
 // Device error word (defined in api.cu).
 unsigned* device_error_word();
