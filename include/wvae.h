@@ -316,6 +316,45 @@ WVAE_API wvae_status wvae_decode_video(const void* const* packed, const float* c
                                        size_t ws_bytes, void* cache, size_t cache_bytes,
                                        int continue_chunk, wvae_stream_t stream);
 
+/* -------------------------------------------------- row-slab decode
+ * One decode split over ranks by latent rows (the FastVideo decoder spreads
+ * one decode over 1-4 GPUs of a node, README "Use" and "Performance and
+ * memory"; the pages do not say how it splits the work).  A rank owns the
+ * latent rows [r0, r0 + rows) and, at stage s, those rows at 2^s times the
+ * resolution; every tensor of its workspace carries its own rows plus one
+ * halo row above and one below.  Before each 3x3 conv the halo rows of the
+ * conv's INPUT (the activation after norm + SiLU: the frame pads with zeros
+ * after the activation) must hold the neighbours' edge rows, or zeros at the
+ * frame's top and bottom.  The library runs the decode one launch at a time
+ * and says where each launch's input lives, so the caller can fill the halo
+ * rows between launches (NCCL point-to-point on the same stream, or copies).
+ * Everything else on the path is per voxel and needs no exchange.
+ *   wvae_decode_rows_steps(): launches per decode (as wvae_decode_trunk).
+ *   wvae_decode_rows_workspace_bytes(T, rows, W, widths): workspace bytes.
+ *   wvae_decode_rows_halo(step, ...): before launch `step`, the tensor whose
+ *     halo rows must be filled: *offset bytes into the workspace, dims =
+ *     {frames, rows + 2 at the stage's resolution, columns, channels}, bf16
+ *     channels-last; dims[0] == 0 when the launch needs no exchange (the
+ *     latent re-layout and conv_in, whose halo comes with the latents).
+ *     Host only: enqueues nothing.
+ *   wvae_decode_rows_step(step, ...): enqueue launch `step` of the decode.
+ *     z_rows: the rank's latents with their halo rows, [1][48][T][rows + 2][W]
+ *     bf16 (rows r0 - 1 .. r0 + rows of the whole latents, zeros outside the
+ *     frame); video_rows: [1][3][T][16 rows][16W] bf16, the rank's video rows.
+ *     Only widths whose last stage has <= 128 channels.
+ * Launching steps 0 .. steps-1 in order, with the halos filled before each,
+ * gives the rank's rows of the whole decode's video.
+ */
+WVAE_API int wvae_decode_rows_steps(void);
+WVAE_API size_t wvae_decode_rows_workspace_bytes(int T, int rows, int W, const int* widths);
+WVAE_API wvae_status wvae_decode_rows_halo(int step, int T, int rows, int W, const int* widths,
+                                           size_t* offset, int* dims);
+WVAE_API wvae_status wvae_decode_rows_step(int step, const void* const* packed,
+                                           const float* const* norms, const void* z_rows,
+                                           void* video_rows, int T, int rows, int W,
+                                           const int* widths, wvae_dtype dtype, void* workspace,
+                                           size_t ws_bytes, wvae_stream_t stream);
+
 /* ------------------------------------------------- res block, no allocation
  * (No counterpart on the pages: this is a convenience of this library.)
  *

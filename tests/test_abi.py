@@ -20,7 +20,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     declared = B.header_symbols()
-    assert len(declared) == 29
+    assert len(declared) == 33
     out = subprocess.check_output(["nm", "-D", "--defined-only", B.LIB_PATH], text=True)
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
     missing = [s for s in declared if s not in exported]

@@ -190,3 +190,44 @@ def test_halo_and_gather_on_a_subgroup():
     assert all(p.exitcode == 0 for p in ps), [p.exitcode for p in ps]
     got = dict(q.get(timeout=10) for _ in range(3))
     assert all(got.values()), got
+
+
+# --------------------------------------------------- the device path's host side
+def test_slab_latents_halo_rows():
+    """A slab's latents: its rows with the neighbouring rows above and below,
+    zeros outside the frame."""
+    z = torch.arange(2 * 3 * 5 * 4, dtype=torch.float32).view(1, 2, 3, 5, 4)
+    top = shard.slab_latents(z, (0, 2))
+    assert top.shape == (1, 2, 3, 4, 4)
+    assert not top[:, :, :, 0].any() and torch.equal(top[:, :, :, 1:], z[:, :, :, 0:3])
+    mid = shard.slab_latents(z, (2, 4))
+    assert torch.equal(mid, z[:, :, :, 1:5])
+    bot = shard.slab_latents(z, (4, 5))
+    assert torch.equal(bot[:, :, :, :2], z[:, :, :, 3:5]) and not bot[:, :, :, 2].any()
+
+
+def test_row_slab_halo_plan():
+    """The library's plan for a slab (host only): the latents' re-layout and
+    conv_in need no exchange; every other launch's input has the stage's own
+    rows plus two, and the four stages' heights and widths follow the
+    upsampling."""
+    import ctypes
+    from video_diffusion_vae_b200 import binding as B
+    lib = B.load()
+    w = (ctypes.c_int * 4)(512, 512, 256, 128)
+    assert lib.wvae_decode_rows_steps() == lib.wvae_decode_trunk_launches() == 22
+    plan = []
+    for i in range(22):
+        off, dims = ctypes.c_size_t(0), (ctypes.c_int * 4)()
+        assert lib.wvae_decode_rows_halo(i, 4, 11, 78, w, ctypes.byref(off), dims) == 0
+        plan.append((off.value, tuple(dims)))
+    assert plan[0][1] == plan[1][1] == (0, 0, 0, 0)
+    stage = {2: 0, 7: 1, 12: 2, 17: 3}
+    for i in range(2, 22):
+        s = max(k for k in stage if k <= i)
+        st = stage[s]
+        assert plan[i][1] == (4, (11 << st) + 2, 78 << st, (512, 512, 256, 128)[st]), (i, plan[i])
+    ws = lib.wvae_decode_rows_workspace_bytes(4, 11, 78, w)
+    assert all(off + 2 * d[0] * d[1] * d[2] * d[3] <= ws for off, d in plan)
+    off, dims = ctypes.c_size_t(0), (ctypes.c_int * 4)()
+    assert lib.wvae_decode_rows_halo(22, 4, 11, 78, w, ctypes.byref(off), dims) == 1

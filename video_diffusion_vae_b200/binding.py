@@ -79,6 +79,12 @@ def load(path: str | None = None):
             "wvae_prepack_conv_winograd": (I, [V, I, V, I, I, V, S, V]),
             "wvae_causal_conv3d_winograd_workspace_bytes": (S, [I, I, I, I, I]),
             "wvae_causal_conv3d_winograd": (I, [V, V, I, I, I, I, I, V, V, V, S, V]),
+            "wvae_decode_rows_steps": (I, []),
+            "wvae_decode_rows_workspace_bytes": (S, [I, I, I, ctypes.POINTER(I)]),
+            "wvae_decode_rows_halo": (I, [I, I, I, I, ctypes.POINTER(I), ctypes.POINTER(S),
+                                          ctypes.POINTER(I)]),
+            "wvae_decode_rows_step": (I, [I, ctypes.POINTER(V), ctypes.POINTER(V), V, V, I, I, I,
+                                          ctypes.POINTER(I), I, V, S, V]),
             "wvae_decode_video_frames": (I, [I, I]),
             "wvae_decode_video_workspace_bytes": (S, [I, I, I, ctypes.POINTER(I)]),
             "wvae_decode_video": (I, [ctypes.POINTER(V), ctypes.POINTER(V), V, V, I, I, I,
@@ -480,6 +486,40 @@ class VideoStream:
         y = _decode_video(z, self.trunk, out, workspace, self.cache, self.started)
         self.started = True
         return y
+
+
+class RowSlab:
+    """One rank's part of a decode split by latent rows (wvae_decode_rows_*):
+    its workspace, and for every launch the view of the tensor whose halo rows
+    must be filled before it (None when the launch needs no exchange)."""
+
+    def __init__(self, trunk: PackedTrunk, T, rows, W, device="cuda"):
+        lib = load()
+        self.trunk, self.T, self.rows, self.W = trunk, T, rows, W
+        self.steps = lib.wvae_decode_rows_steps()
+        n = lib.wvae_decode_rows_workspace_bytes(T, rows, W, trunk._widths_arr)
+        if n == 0:
+            raise ValueError("unsupported row slab")
+        self.ws = _workspace(n, torch.device(device))
+        self.halo = []
+        for i in range(self.steps):
+            off = ctypes.c_size_t(0)
+            dims = (ctypes.c_int * 4)()
+            _check("wvae_decode_rows_halo", lib.wvae_decode_rows_halo(
+                i, T, rows, W, trunk._widths_arr, ctypes.byref(off), dims))
+            if dims[0] == 0:
+                self.halo.append(None)
+                continue
+            nel = dims[0] * dims[1] * dims[2] * dims[3]
+            flat = self.ws[off.value:off.value + 2 * nel].view(torch.bfloat16)
+            self.halo.append(flat.view(dims[0], dims[1], dims[2], dims[3]))
+
+    def step(self, i, z_rows, video_rows):
+        """Enqueue launch i (z_rows [1, 48, T, rows + 2, W], video_rows [1, 3, T, 16 rows, 16 W])."""
+        tr = self.trunk
+        _check("wvae_decode_rows_step", load().wvae_decode_rows_step(
+            i, tr._packed_arr, tr._norm_arr, _ptr(z_rows), _ptr(video_rows), self.T, self.rows,
+            self.W, tr._widths_arr, BF16, _ptr(self.ws), _nbytes(self.ws), _stream()))
 
 
 class TrunkGraph:

@@ -165,6 +165,7 @@ struct TcConv {
   int phases = 1;            // 4: upsample-conv phase mode (packed by prepack_upsample)
   int tdup = 0;              // phase mode: temporal 2x copies of the output (ConvParams::tdup)
   int wino = 0;              // Winograd products over the 16 transform planes (ConvParams::wino)
+  int out_row0 = 0, out_rows = 0;  // phase mode: output row window (ConvParams)
   ConvEpilogue ep{};
 };
 
@@ -199,6 +200,8 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   p.phases = a.phases;
   p.tdup = a.phases == 4 ? a.tdup : 0;
   p.wino = a.wino;
+  p.out_row0 = a.phases == 4 ? a.out_row0 : 0;
+  p.out_rows = a.phases == 4 ? a.out_rows : 0;
   p.has_cache = a.cache != nullptr;
   // The fused norm needs every output channel of a voxel: one CTA holds them
   // all (BN = Cout) up to 256; at 512 a cluster of two CTAs splits N and swaps
@@ -733,8 +736,8 @@ struct TrunkBuffers {
   size_t total;
 };
 
-// F: frames per stage (T everywhere without temporal upsampling).
-TrunkBuffers trunk_buffers(const int* F, int H, int W, const int* C) {
+// F, Hs, Ws: frames, rows and columns per stage.
+TrunkBuffers trunk_buffers(const int* F, const int* Hs, const int* Ws, const int* C) {
   TrunkBuffers b;
   size_t off = 0;
   auto take = [&](size_t n) {
@@ -742,10 +745,10 @@ TrunkBuffers trunk_buffers(const int* F, int H, int W, const int* C) {
     off += round_up_sz(n, 256);
     return o;
   };
-  const size_t v0 = static_cast<size_t>(F[0]) * H * W;
+  const size_t v0 = static_cast<size_t>(F[0]) * Hs[0] * Ws[0];
   size_t max_h = 0, max_act = 0, max_up = 0;
   for (int s = 0; s < 4; ++s) {
-    const size_t vs = (static_cast<size_t>(F[s]) * H * W) << (2 * s);
+    const size_t vs = static_cast<size_t>(F[s]) * Hs[s] * Ws[s];
     max_h = std::max(max_h, vs * C[s] * 4);
     max_act = std::max(max_act, vs * C[s] * 2);
     if (s < 3) max_up = std::max(max_up, vs * C[s] * 2);
@@ -807,7 +810,8 @@ size_t wvae_decode_trunk_workspace_bytes(int T, int H, int W, const int* widths)
   for (int s = 0; s < 4; ++s)
     if (C[s] < 64) return 0;
   const int F[4] = {T, T, T, T};
-  return trunk_buffers(F, H, W, C).total;
+  const int Hs[4] = {H, 2 * H, 4 * H, 8 * H}, Ws[4] = {W, 2 * W, 4 * W, 8 * W};
+  return trunk_buffers(F, Hs, Ws, C).total;
 }
 
 int wvae_decode_video_frames(int T, int continue_chunk) {
@@ -821,65 +825,136 @@ size_t wvae_decode_video_workspace_bytes(int T, int H, int W, const int* widths)
   for (int s = 0; s < 4; ++s)
     if (C[s] < 64) return 0;
   const int F[4] = {T, 2 * T, 4 * T, 4 * T};  // a continuing chunk's counts bound the first's
-  return trunk_buffers(F, H, W, C).total;
+  const int Hs[4] = {H, 2 * H, 4 * H, 8 * H}, Ws[4] = {W, 2 * W, 4 * W, 8 * W};
+  return trunk_buffers(F, Hs, Ws, C).total;
+}
+
+// Row slab: every stage carries its own rows plus a halo row above and below.
+size_t wvae_decode_rows_workspace_bytes(int T, int rows, int W, const int* widths) {
+  if (T < 1 || rows < 1 || W < 1) return 0;
+  const int* C = widths ? widths : kDefaultWidths;
+  for (int s = 0; s < 4; ++s)
+    if (C[s] < 64) return 0;
+  const int F[4] = {T, T, T, T};
+  const int Hs[4] = {rows + 2, 2 * rows + 2, 4 * rows + 2, 8 * rows + 2};
+  const int Ws[4] = {W, 2 * W, 4 * W, 8 * W};
+  return trunk_buffers(F, Hs, Ws, C).total;
 }
 
 namespace {
 constexpr int kTrunkLaunches = 22;
 
-// cache (optional): the causal caches of a chunked decode; continue_chunk:
-// read the front frames from it (else zeros); it is rewritten with this
-// chunk's last two input frames of every causal conv.
+// Where the input of one launch of a row-slab decode lives in the workspace
+// (the tensor whose halo rows the caller refreshes before that launch).
+struct HaloQuery {
+  int step = -1;
+  int found = 0;
+  size_t offset = 0;
+  int dims[4] = {0, 0, 0, 0};  // frames, rows (own + 2 halo), columns, channels; bf16
+};
+
+// How a decode runs: per-launch events, causal caches of a chunked decode
+// (continue_chunk: read the front frames from them, else zeros; they are
+// rewritten with this chunk's last two input frames of every causal conv),
+// temporal upsampling, a row slab, one launch only, or a halo query.
+struct TrunkRun {
+  void* const* events = nullptr;
+  int n_events = 0;
+  void* cache = nullptr;
+  size_t cache_bytes = 0;
+  int continue_chunk = 0;
+  int temporal = 0;
+  int rows = 0;            // > 0: a slab of `rows` latent rows (H == rows), one halo row
+                           // above and below at every stage
+  int only_step = -1;      // >= 0: enqueue launch `only_step` alone
+  HaloQuery* query = nullptr;  // enqueue nothing; describe query->step's input
+};
+
 wvae_status decode_trunk_impl(const void* const* packed, const float* const* norms, const void* z,
                               void* video, int T, int H, int W, const int* widths,
                               wvae_dtype dtype, void* workspace, size_t ws_bytes,
-                              void* const* events, int n_events, void* cache, size_t cache_bytes,
-                              int continue_chunk, int temporal, wvae_stream_t stream) {
-  if (!packed || !norms || !z || !video || !workspace) return WVAE_ERR_INVALID_ARG;
+                              const TrunkRun& run, wvae_stream_t stream) {
+  void* const* events = run.events;
+  void* cache = run.cache;
+  const int continue_chunk = run.continue_chunk;
+  const bool query = run.query != nullptr;
+  const bool slab = run.rows > 0;
+  if (!query && (!packed || !norms || !z || !video || !workspace)) return WVAE_ERR_INVALID_ARG;
   if (cache != nullptr && T < 2) return WVAE_ERR_INVALID_ARG;  // the cache holds two frames
-  if (events != nullptr && n_events < 2 * kTrunkLaunches) return WVAE_ERR_INVALID_ARG;
+  if (events != nullptr && run.n_events < 2 * kTrunkLaunches) return WVAE_ERR_INVALID_ARG;
   if (T < 1 || H < 1 || W < 1) return WVAE_ERR_INVALID_ARG;
+  if (slab && (cache != nullptr || run.temporal)) return WVAE_ERR_UNSUPPORTED;
+  if (run.only_step >= kTrunkLaunches) return WVAE_ERR_INVALID_ARG;
   if (dtype != WVAE_BF16) return WVAE_ERR_UNSUPPORTED;
   const int* C = widths ? widths : kDefaultWidths;
   for (int s = 0; s < 4; ++s)
     if (C[s] % 64 != 0 || !bf16_cout_ok(C[s])) return WVAE_ERR_UNSUPPORTED;
-  for (int i = 0; i < 21; ++i)
-    if (!packed[i]) return WVAE_ERR_INVALID_ARG;
-  for (int i = 0; i < 34; ++i)
-    if (!norms[i]) return WVAE_ERR_INVALID_ARG;
-  for (int i = 0; i < 21; ++i)
-    if (!a16(packed[i])) return WVAE_ERR_ALIGNMENT;
-  if (!a16(z) || !a16(video) || !a16(workspace)) return WVAE_ERR_ALIGNMENT;
+  if (!query) {
+    for (int i = 0; i < 21; ++i)
+      if (!packed[i]) return WVAE_ERR_INVALID_ARG;
+    for (int i = 0; i < 34; ++i)
+      if (!norms[i]) return WVAE_ERR_INVALID_ARG;
+    for (int i = 0; i < 21; ++i)
+      if (!a16(packed[i])) return WVAE_ERR_ALIGNMENT;
+    if (!a16(z) || !a16(video) || !a16(workspace)) return WVAE_ERR_ALIGNMENT;
+  }
   if (continue_chunk && cache == nullptr) return WVAE_ERR_INVALID_ARG;
   // Frames per stage: with temporal upsampling the upsample convs of stages 0
   // and 1 also double the frames (the decode's first frame once).
   const bool first = !continue_chunk;
   int F[4] = {T, T, T, T};
-  if (temporal) {
+  if (run.temporal) {
     F[1] = first ? 2 * T - 1 : 2 * T;
     F[2] = first ? 2 * F[1] - 1 : 2 * F[1];
     F[3] = F[2];
   }
-  const TrunkBuffers B = trunk_buffers(F, H, W, C);
-  if (ws_bytes < B.total) return WVAE_ERR_WORKSPACE;
+  // Rows and columns per stage; a slab's tensors carry a halo row on each side.
+  int HS[4], WS[4];
+  for (int s2 = 0; s2 < 4; ++s2) {
+    HS[s2] = slab ? (run.rows << s2) + 2 : H << s2;
+    WS[s2] = W << s2;
+  }
+  const TrunkBuffers B = trunk_buffers(F, HS, WS, C);
+  if (!query && ws_bytes < B.total) return WVAE_ERR_WORKSPACE;
   const TrunkCaches K = trunk_caches(H, W, C);
   if (cache != nullptr) {
     if (!a16(cache)) return WVAE_ERR_ALIGNMENT;
-    if (cache_bytes < K.total) return WVAE_ERR_WORKSPACE;
+    if (run.cache_bytes < K.total) return WVAE_ERR_WORKSPACE;
   }
   DeviceInfo* d = nullptr;
-  wvae_status st = device_info(&d);
-  if (st != WVAE_OK) return st;
+  if (!query) {
+    wvae_status st0 = device_info(&d);
+    if (st0 != WVAE_OK) return st0;
+  }
+  wvae_status st = WVAE_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int launch = 0;
+  // whether launch `launch` is enqueued by this call
+  auto exec = [&]() { return !query && (run.only_step < 0 || run.only_step == launch); };
   auto mark = [&](int which) {
-    if (events != nullptr)
+    if (events != nullptr && exec())
       cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[2 * launch + which]), s);
   };
+  char* ws = static_cast<char*>(workspace);
+  // the input of a 3x3 conv whose halo a slab's caller refreshes
+  auto note_input = [&](const void* x, int t, int hh, int ww, int cc) {
+    if (query && run.query->step == launch) {
+      run.query->found = 1;
+      run.query->offset = static_cast<size_t>(static_cast<const char*>(x) - ws);
+      run.query->dims[0] = t;
+      run.query->dims[1] = hh;
+      run.query->dims[2] = ww;
+      run.query->dims[3] = cc;
+    }
+  };
   auto conv = [&](const TcConv& c) {
-    mark(0);
-    wvae_status r = run_tc_conv(*d, c, s);
-    mark(1);
+    if (slab && launch > 1) note_input(c.x, c.T, c.H, c.W, c.cin_pad);
+    wvae_status r = WVAE_OK;
+    if (exec()) {
+      mark(0);
+      r = run_tc_conv(*d, c, s);
+      mark(1);
+    }
     ++launch;
     return r;
   };
@@ -896,36 +971,39 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
     return cuda_status(cudaMemcpyAsync(entry, static_cast<const char*>(c.x) + (c.T - 2) * frame,
                                        2 * frame, cudaMemcpyDeviceToDevice, s));
   };
-  char* ws = static_cast<char*>(workspace);
   void* zcl = ws + B.zcl;
   float* h = reinterpret_cast<float*>(ws + B.h);
   __nv_bfloat16* act[2] = {reinterpret_cast<__nv_bfloat16*>(ws + B.act1),
                            reinterpret_cast<__nv_bfloat16*>(ws + B.act2)};
   void* up = ws + B.up;
 
-  // latents NCDHW -> channels-last, channels padded 48 -> 64
-  mark(0);
-  st = cuda_status(launch_ncdhw_to_cl_pad(static_cast<const __nv_bfloat16*>(z),
-                                          static_cast<__nv_bfloat16*>(zcl), kZChannels, kZPad, T,
-                                          H, W, s));
-  mark(1);
+  // latents NCDHW -> channels-last, channels padded 48 -> 64 (a slab's latents
+  // come with their halo rows: the caller reads them from the whole latents)
+  if (exec()) {
+    mark(0);
+    st = cuda_status(launch_ncdhw_to_cl_pad(static_cast<const __nv_bfloat16*>(z),
+                                            static_cast<__nv_bfloat16*>(zcl), kZChannels, kZPad, T,
+                                            HS[0], W, s));
+    mark(1);
+  }
   ++launch;
   if (st != WVAE_OK) return st;
 
   int pi = 0, ni = 0;
   auto next_norm = [&](const float** g, const float** b) {
-    *g = norms[2 * ni];
-    *b = norms[2 * ni + 1];
+    *g = norms ? norms[2 * ni] : nullptr;
+    *b = norms ? norms[2 * ni + 1] : nullptr;
     ++ni;
   };
-  int Hs = H, Ws = W;
+  auto next_packed = [&]() { return packed ? packed[pi++] : (++pi, nullptr); };
+  int Hs = HS[0], Ws = W;
 
   // conv_in: residual stream h (fp32) + A1 of stage 0, block 0.
   {
     TcConv c;
     c.x = zcl;
     c.cin_pad = kZPad;
-    c.packed = packed[pi++];
+    c.packed = next_packed();
     c.cout = C[0];
     c.T = T; c.H = Hs; c.W = Ws;
     c.ep.out = h;
@@ -933,7 +1011,7 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
     c.ep.act = act[0];
     next_norm(&c.ep.gamma, &c.ep.beta);
     c.ep.eps = 1e-12f;
-    st = causal_conv(c, static_cast<size_t>(H) * W * kZPad * 2);
+    st = causal_conv(c, static_cast<size_t>(Hs) * W * kZPad * 2);
     if (st != WVAE_OK) return st;
   }
   for (int stg = 0; stg < 4; ++stg) {
@@ -945,7 +1023,7 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
       TcConv c1;
       c1.x = act[0];
       c1.cin_pad = Cs;
-      c1.packed = packed[pi++];
+      c1.packed = next_packed();
       c1.cout = Cs;
       c1.T = Ts; c1.H = Hs; c1.W = Ws;
       c1.ep.act = act[1];
@@ -957,7 +1035,7 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
       TcConv c2;
       c2.x = act[1];
       c2.cin_pad = Cs;
-      c2.packed = packed[pi++];
+      c2.packed = next_packed();
       c2.cout = Cs;
       c2.T = Ts; c2.H = Hs; c2.W = Ws;
       c2.ep.residual = h;
@@ -987,12 +1065,18 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
       TcConv cu;
       cu.x = up;
       cu.cin_pad = Cs;
-      cu.packed = packed[pi++];
+      cu.packed = next_packed();
       cu.cout = C[stg + 1];
       cu.T = Ts; cu.H = Hs; cu.W = Ws;
       cu.phases = 4;
       if (F[stg + 1] != Ts) cu.tdup = first ? 1 : 2;
-      Hs *= 2;
+      if (slab) {
+        // output row 2h + p' of the halo-extended input is row 2h + p' - 1 of the
+        // next stage's slab (its own rows and one halo row each side)
+        cu.out_row0 = 1;
+        cu.out_rows = HS[stg + 1];
+      }
+      Hs = HS[stg + 1];
       Ws *= 2;
       cu.ep.out = h;
       cu.ep.out_f32 = 1;
@@ -1008,41 +1092,47 @@ wvae_status decode_trunk_impl(const void* const* packed, const float* const* nor
   if (C[3] <= 128) {
     char* entry = cache != nullptr ? static_cast<char*>(cache) + K.off[ck] : nullptr;
     ++ck;
-    HeadParams hp;
-    std::memset(&hp, 0, sizeof(hp));
-    const PackedLayout L = packed_layout(kHeadOut, C[3], 3, 3, 3, WVAE_BF16);
-    if (!encode_act(&hp.tmA, act[0], C[3], Ws, Hs, F[3], kHeadTileCols, kHeadTileRows + 2))
-      return WVAE_ERR_CUDA;
-    if (entry != nullptr && continue_chunk) {
-      if (!encode_act(&hp.tmC, entry, C[3], Ws, Hs, 2, kHeadTileCols, kHeadTileRows + 2))
+    if (slab) note_input(act[0], F[3], Hs, Ws, C[3]);
+    const void* pk = next_packed();
+    if (exec()) {
+      HeadParams hp;
+      std::memset(&hp, 0, sizeof(hp));
+      const PackedLayout L = packed_layout(kHeadOut, C[3], 3, 3, 3, WVAE_BF16);
+      if (!encode_act(&hp.tmA, act[0], C[3], Ws, Hs, F[3], kHeadTileCols, kHeadTileRows + 2))
         return WVAE_ERR_CUDA;
-      hp.has_cache = 1;
+      if (entry != nullptr && continue_chunk) {
+        if (!encode_act(&hp.tmC, entry, C[3], Ws, Hs, 2, kHeadTileCols, kHeadTileRows + 2))
+          return WVAE_ERR_CUDA;
+        hp.has_cache = 1;
+      }
+      if (!encode_weights(&hp.tmB, pk, L.taps * C[3], L.cout_pad, 16)) return WVAE_ERR_CUDA;
+      hp.bias = reinterpret_cast<const float*>(static_cast<const char*>(pk) + L.bias_off);
+      hp.video = static_cast<__nv_bfloat16*>(video);
+      hp.T = F[3];
+      hp.H = Hs;
+      hp.W = Ws;
+      hp.cin = C[3];
+      hp.row0 = slab ? 1 : 0;
+      hp.rows_out = slab ? Hs - 2 : Hs;
+      hp.tiles_w = (Ws + kHeadOutCols - 1) / kHeadOutCols;
+      hp.tiles_h = (Hs + kHeadTileRows - 1) / kHeadTileRows;
+      hp.num_tiles = hp.tiles_w * hp.tiles_h;
+      hp.err = d->err;
+      mark(0);
+      st = cuda_status(launch_head_tc(hp, d->num_sms, s));
+      mark(1);
     }
-    const void* pk = packed[pi++];
-    if (!encode_weights(&hp.tmB, pk, L.taps * C[3], L.cout_pad, 16)) return WVAE_ERR_CUDA;
-    hp.bias = reinterpret_cast<const float*>(static_cast<const char*>(pk) + L.bias_off);
-    hp.video = static_cast<__nv_bfloat16*>(video);
-    hp.T = F[3];
-    hp.H = Hs;
-    hp.W = Ws;
-    hp.cin = C[3];
-    hp.tiles_w = (Ws + kHeadOutCols - 1) / kHeadOutCols;
-    hp.tiles_h = (Hs + kHeadTileRows - 1) / kHeadTileRows;
-    hp.num_tiles = hp.tiles_w * hp.tiles_h;
-    hp.err = d->err;
-    mark(0);
-    st = cuda_status(launch_head_tc(hp, d->num_sms, s));
-    mark(1);
     ++launch;
-    if (st != WVAE_OK || entry == nullptr) return st;
+    if (st != WVAE_OK || entry == nullptr || query) return st;
     const size_t frame = static_cast<size_t>(Hs) * Ws * C[3] * 2;
     return cuda_status(cudaMemcpyAsync(entry, reinterpret_cast<const char*>(act[0]) + (F[3] - 2) * frame,
                                        2 * frame, cudaMemcpyDeviceToDevice, s));
   }
+  if (slab) return WVAE_ERR_UNSUPPORTED;  // the slab's head needs the head kernel (C3 <= 128)
   TcConv ch;
   ch.x = act[0];
   ch.cin_pad = C[3];
-  ch.packed = packed[pi++];
+  ch.packed = next_packed();
   ch.cout = kHeadOut;
   ch.T = F[3]; ch.H = Hs; ch.W = Ws;
   ch.ep.video = static_cast<__nv_bfloat16*>(video);
@@ -1057,7 +1147,7 @@ wvae_status wvae_decode_trunk(const void* const* packed, const float* const* nor
                               wvae_dtype dtype, void* workspace, size_t ws_bytes,
                               wvae_stream_t stream) {
   return decode_trunk_impl(packed, norms, z, video, T, H, W, widths, dtype, workspace, ws_bytes,
-                           nullptr, 0, nullptr, 0, 0, 0, stream);
+                           TrunkRun{}, stream);
 }
 
 wvae_status wvae_decode_trunk_chunk(const void* const* packed, const float* const* norms,
@@ -1066,8 +1156,12 @@ wvae_status wvae_decode_trunk_chunk(const void* const* packed, const float* cons
                                     size_t ws_bytes, void* cache, size_t cache_bytes,
                                     int continue_chunk, wvae_stream_t stream) {
   if (cache == nullptr) return WVAE_ERR_INVALID_ARG;
+  TrunkRun run;
+  run.cache = cache;
+  run.cache_bytes = cache_bytes;
+  run.continue_chunk = continue_chunk;
   return decode_trunk_impl(packed, norms, z, video, T, H, W, widths, dtype, workspace, ws_bytes,
-                           nullptr, 0, cache, cache_bytes, continue_chunk, 0, stream);
+                           run, stream);
 }
 
 wvae_status wvae_decode_video(const void* const* packed, const float* const* norms, const void* z,
@@ -1075,8 +1169,43 @@ wvae_status wvae_decode_video(const void* const* packed, const float* const* nor
                               wvae_dtype dtype, void* workspace, size_t ws_bytes, void* cache,
                               size_t cache_bytes, int continue_chunk, wvae_stream_t stream) {
   if (cache == nullptr && continue_chunk) return WVAE_ERR_INVALID_ARG;
+  TrunkRun run;
+  run.cache = cache;
+  run.cache_bytes = cache_bytes;
+  run.continue_chunk = continue_chunk;
+  run.temporal = 1;
   return decode_trunk_impl(packed, norms, z, video, T, H, W, widths, dtype, workspace, ws_bytes,
-                           nullptr, 0, cache, cache_bytes, continue_chunk, 1, stream);
+                           run, stream);
+}
+
+int wvae_decode_rows_steps(void) { return kTrunkLaunches; }
+
+wvae_status wvae_decode_rows_halo(int step, int T, int rows, int W, const int* widths,
+                                  size_t* offset, int* dims) {
+  if (!offset || !dims || step < 0 || step >= kTrunkLaunches) return WVAE_ERR_INVALID_ARG;
+  HaloQuery q;
+  q.step = step;
+  TrunkRun run;
+  run.rows = rows;
+  run.query = &q;
+  const wvae_status st = decode_trunk_impl(nullptr, nullptr, nullptr, nullptr, T, rows, W, widths,
+                                           WVAE_BF16, nullptr, 0, run, nullptr);
+  if (st != WVAE_OK) return st;
+  *offset = q.found ? q.offset : 0;
+  for (int i = 0; i < 4; ++i) dims[i] = q.found ? q.dims[i] : 0;
+  return WVAE_OK;
+}
+
+wvae_status wvae_decode_rows_step(int step, const void* const* packed, const float* const* norms,
+                                  const void* z_rows, void* video_rows, int T, int rows, int W,
+                                  const int* widths, wvae_dtype dtype, void* workspace,
+                                  size_t ws_bytes, wvae_stream_t stream) {
+  if (step < 0 || step >= kTrunkLaunches) return WVAE_ERR_INVALID_ARG;
+  TrunkRun run;
+  run.rows = rows;
+  run.only_step = step;
+  return decode_trunk_impl(packed, norms, z_rows, video_rows, T, rows, W, widths, dtype, workspace,
+                           ws_bytes, run, stream);
 }
 
 wvae_status wvae_decode_trunk_timed(const void* const* packed, const float* const* norms,
@@ -1085,8 +1214,11 @@ wvae_status wvae_decode_trunk_timed(const void* const* packed, const float* cons
                                     size_t ws_bytes, void* const* events, int n_events,
                                     wvae_stream_t stream) {
   if (events == nullptr) return WVAE_ERR_INVALID_ARG;
+  TrunkRun run;
+  run.events = events;
+  run.n_events = n_events;
   return decode_trunk_impl(packed, norms, z, video, T, H, W, widths, dtype, workspace, ws_bytes,
-                           events, n_events, nullptr, 0, 0, 0, stream);
+                           run, stream);
 }
 
 // ------------------------------------------------- res block, no allocation

@@ -789,7 +789,12 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
       const int c = idx % p.tile_cols;
       const int h = tc.th * p.tile_rows + idx / p.tile_cols;
       const int w = tc.tw * p.out_cols + c - (p.nw > 1 ? 1 : 0);
-      const bool valid = h < p.H && w < p.W && (p.nw == 1 || (c >= 1 && c <= p.tile_cols - 2));
+      // phase mode with a row window (out_rows > 0): output row 2h + p' lands at row
+      // 2h + p' - out_row0 of an out_rows-row output, or nowhere
+      const int ho = p.phases == 4 ? 2 * h + (tc.phase >> 1) - p.out_row0 : h;
+      const int Ho = p.out_rows > 0 ? p.out_rows : 2 * p.H;
+      const bool valid = h < p.H && w < p.W && (p.nw == 1 || (c >= 1 && c <= p.tile_cols - 2)) &&
+                         (p.out_rows == 0 || (ho >= 0 && ho < p.out_rows));
       // output voxel: (t, h, w), or (t, 2h + p', 2w + q') of the 2H x 2W output in phase
       // mode.  With a temporal 2x step (phase mode only) input frame t goes to output
       // frames 2t - 1 and 2t (tdup 1: frame 0 of the decode once), or 2t and 2t + 1
@@ -805,8 +810,7 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
       auto out_vox = [&](int to) {
         if (p.wino)  // transform plane xi = phase of the products
           return ((static_cast<size_t>(tc.phase) * p.T + to) * p.H + h) * p.W + w;
-        return p.phases == 4 ? (static_cast<size_t>(to) * 2 * p.H + 2 * h + (tc.phase >> 1)) *
-                                       (2 * p.W) + 2 * w + (tc.phase & 1)
+        return p.phases == 4 ? (static_cast<size_t>(to) * Ho + ho) * (2 * p.W) + 2 * w + (tc.phase & 1)
                              : (static_cast<size_t>(to) * p.H + h) * p.W + w;
       };
       const size_t vox = out_vox(t0);

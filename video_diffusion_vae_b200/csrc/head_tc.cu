@@ -205,13 +205,17 @@ __device__ void head_epilogue(const HeadParams& p, const HeadSmem& s, uint32_t t
 #pragma unroll
   for (int o = 0; o < 12; ++o) bias[o] = p.bias[o];
   const int f0 = p.has_cache ? -2 : 0;
-  const size_t H2 = 2 * static_cast<size_t>(p.H), W2 = 2 * static_cast<size_t>(p.W);
+  // video rows: 2 (h - row0) + i for the rows_out rows from row0 on
+  const int rows_out = p.rows_out > 0 ? p.rows_out : p.H;
+  const size_t H2 = 2 * static_cast<size_t>(rows_out), W2 = 2 * static_cast<size_t>(p.W);
   uint32_t it = 0;
   for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
     int h0, w0;
     head_tile(p, tile, h0, w0);
     const int h = h0 + r, w = w0 - 1 + c;
-    const bool valid = h < p.H && c >= 1 && c <= kCols - 2 && w < p.W;
+    const bool valid = h < p.H && c >= 1 && c <= kCols - 2 && w < p.W && h >= p.row0 &&
+                       h < p.row0 + rows_out;
+    const int hv = h - p.row0;
     float pend_a[16], pend_b[16];     // partial sums of output frames f and f + 1
 #pragma unroll
     for (int o = 0; o < 16; ++o) pend_a[o] = pend_b[o] = 0.0f;
@@ -245,7 +249,7 @@ __device__ void head_epilogue(const HeadParams& p, const HeadSmem& s, uint32_t t
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             const int o = 4 * cv + 2 * i;
-            const size_t off = ((static_cast<size_t>(cv) * p.T + f) * H2 + 2 * h + i) * W2 + 2 * w;
+            const size_t off = ((static_cast<size_t>(cv) * p.T + f) * H2 + 2 * hv + i) * W2 + 2 * w;
             *reinterpret_cast<uint32_t*>(p.video + off) =
                 pack_bf16x2(out[o] + bias[o], out[o + 1] + bias[o + 1]);
           }

@@ -55,6 +55,8 @@ struct ConvParams {
   int wino;          // 1: Winograd products: phases = 16 transform planes, fp16 operands, A
                      //    = the planes [16][T][H][W][cin] (tmA 5-D, H x W = the tile grid),
                      //    weights [cout_pad][16 x KT][cin_pad], out [16][T][H][W][cout]
+  int out_row0, out_rows;  // phase mode: output row 2h + p' is written at row 2h + p' - out_row0
+                           //    of an out_rows-row output, if inside it (out_rows 0: 2H rows)
   int tdup;          // phase mode: a temporal 2x step in the output frames (1: input frame
                      //    t -> 2t - 1 and 2t, frame 0 once; 2: t -> 2t and 2t + 1)
   int nsplit;        // 2: a cluster of 2 CTAs splits N (rank = N tile) and exchanges the
@@ -161,6 +163,8 @@ struct HeadParams {
   int T, H, W, cin;
   int tiles_w, tiles_h, num_tiles;
   int has_cache;     // frames -2, -1 come from tmC
+  int row0, rows_out;  // video rows 2 (h - row0) + i for rows h in [row0, row0 + rows_out)
+                       // (rows_out 0: all H rows, row0 0)
   unsigned* err;
 };
 size_t head_tc_smem_bytes(int cin);

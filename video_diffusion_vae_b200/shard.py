@@ -24,6 +24,13 @@ With the extra rows in place a conv computed over rows + 2 rows gives its own
 rows exactly (the two outer rows are discarded, or overwritten by the next
 exchange), so the convs themselves need no change.  Works on CPU tensors
 (gloo) and CUDA tensors (NCCL) alike.
+
+On the device (decode_rows): the library's row-slab decode keeps every
+tensor with one halo row per side and runs one launch at a time
+(wvae_decode_rows_*); between launches the caller fills the halo rows of the
+next conv's input.  The upsample convs write the next stage's slab (own rows
+plus one halo row each side) directly, and the head writes the rank's own
+video rows.
 """
 from __future__ import annotations
 
@@ -118,3 +125,67 @@ def gather_rows(mine: torch.Tensor, parts: list[tuple[int, int]], scale: int, ra
         dist.recv(buf, _peer(group, src), group)
         pieces.append(buf)
     return torch.cat(pieces, dim=row_dim)
+
+
+# ------------------------------------------------------------ device decode
+def slab_latents(z: torch.Tensor, part: tuple[int, int]) -> torch.Tensor:
+    """The latents of a rank's rows with one halo row above and below, taken
+    from the whole latents z [1, C, T, H, W] (zeros outside the frame)."""
+    r0, r1 = part
+    H = z.shape[3]
+    out = z.new_zeros(z.shape[:3] + (r1 - r0 + 2,) + z.shape[4:])
+    a, b = max(r0 - 1, 0), min(r1 + 1, H)
+    out[:, :, :, a - (r0 - 1):b - (r0 - 1)] = z[:, :, :, a:b]
+    return out.contiguous()
+
+
+def decode_rows(z, trunk, rank: int, world: int, group=None, gather: bool = True):
+    """One decode split over the ranks of `group` by latent rows (every rank
+    passes the same latents z [1, 48, T, H, W], bf16, on its GPU).  Each rank
+    decodes its rows through the library's row-slab steps, exchanging the
+    halo rows of every 3x3 conv's input with its neighbours (NCCL point-to-
+    point for CUDA tensors).  Returns the whole video on rank 0 (gather=True,
+    as the pages' decoder does) or this rank's video rows."""
+    from video_diffusion_vae_b200 import binding as B
+    _, _, T, H, W = z.shape
+    parts = partition(H, world)
+    r0, r1 = parts[rank]
+    slab = B.RowSlab(trunk, T, r1 - r0, W, device=z.device)
+    zr = slab_latents(z, (r0, r1))
+    video = torch.empty((1, 3, T, 16 * (r1 - r0), 16 * W), dtype=torch.bfloat16, device=z.device)
+    for i in range(slab.steps):
+        if slab.halo[i] is not None:
+            exchange_halo(slab.halo[i], rank, world, 1, group)
+        slab.step(i, zr, video)
+    if not gather:
+        return video
+    return gather_rows(video, parts, 16, rank, world, 3, group)
+
+
+def decode_rows_emulated(z, trunk, world: int):
+    """The row split on one device: `world` slabs step in lockstep and the halo
+    rows are copied between them (standing in for the NCCL exchange).
+    Returns the assembled video."""
+    from video_diffusion_vae_b200 import binding as B
+    _, _, T, H, W = z.shape
+    parts = partition(H, world)
+    slabs = [B.RowSlab(trunk, T, r1 - r0, W, device=z.device) for r0, r1 in parts]
+    zs = [slab_latents(z, p) for p in parts]
+    videos = [torch.empty((1, 3, T, 16 * (r1 - r0), 16 * W), dtype=torch.bfloat16, device=z.device)
+              for r0, r1 in parts]
+    for i in range(slabs[0].steps):
+        views = [sl.halo[i] for sl in slabs]
+        if views[0] is not None:
+            for r, v in enumerate(views):
+                n = v.shape[1]
+                if r > 0:
+                    v[:, 0].copy_(views[r - 1][:, views[r - 1].shape[1] - 2])
+                else:
+                    v[:, 0].zero_()
+                if r < world - 1:
+                    v[:, n - 1].copy_(views[r + 1][:, 1])
+                else:
+                    v[:, n - 1].zero_()
+        for sl, zr, vd in zip(slabs, zs, videos):
+            sl.step(i, zr, vd)
+    return torch.cat(videos, dim=3)
