@@ -464,8 +464,9 @@ def profile_case(name: str, launches: int = 3) -> int:
     """Run one kernel workload `launches` times (for an ncu capture; no JSON line).
     conv512: causal conv 512->512 on [4,88,156]; norm512 / norm256: norm-SiLU on
     [512,4,88,156] / [256,4,176,312]; res256: res block 256->256 on [4,176,312];
-    res128: res block 128->128 on [4,352,624] (the last stage's shape); trunk:
-    one trunk decode."""
+    res128: res block 128->128 on [4,352,624] (the last stage's shape); wino512 /
+    wino256: the Winograd conv 512->512 on [4,88,156] / 256->256 on [4,176,312];
+    trunk: one trunk decode."""
     import torch
     from video_diffusion_vae_b200 import binding as B
     from video_diffusion_vae_b200 import synth
@@ -491,6 +492,12 @@ def profile_case(name: str, launches: int = 3) -> int:
         blk = B.PackedResBlock(p)
         xd = x.permute(1, 2, 3, 0).contiguous().cuda().bfloat16()
         fn = lambda: B.resblock(xd, blk)  # noqa: E731
+    elif name in ("wino512", "wino256"):
+        c, Hh, Ww = (512, 88, 156) if name == "wino512" else (256, 176, 312)
+        x, w, b = synth.conv_input(cin=c, cout=c, T=4, H=Hh, W=Ww, seed=0)
+        pw = B.prepack_conv_winograd(w.cuda().bfloat16(), b.cuda())
+        xd = x.permute(1, 2, 3, 0).contiguous().cuda().bfloat16()
+        fn = lambda: B.causal_conv3d_winograd(xd, pw)  # noqa: E731
     elif name == "trunk":
         z, params = synth.trunk_input()
         tr = B.PackedTrunk(params)
@@ -516,7 +523,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", default=None,
                     help="run one kernel workload for an ncu capture (conv512, norm512, norm256, "
-                         "res256, res128, trunk) and exit")
+                         "res256, res128, wino512, wino256, trunk) and exit")
     args = ap.parse_args()
     if args.profile_case:
         return profile_case(args.profile_case)
