@@ -139,3 +139,25 @@ def test_conv_epilogue_16_byte_aligned_buffers():
     torch.cuda.synchronize()
     assert torch.equal(out16, y32)
     assert_close(from_cl(y32), O.causal_conv3d(x, w, b) + res.double().numpy(), torch.bfloat16, "res")
+
+
+@pytest.mark.parametrize("cout", [128, 64])
+def test_conv_many_waves_sampled(cout):
+    """128 -> 128 and 64 -> 64 on [cin, 4, 256, 320]: 1,280 CTA tiles of 16 x 16
+    voxels over the 148 SMs (8.6 waves; two accumulators alternate), ragged
+    nowhere.  512 sampled voxels (corners, edges, tile and sub-tile seams)
+    against the oracle."""
+    T, H, W = 4, 256, 320
+    x, w, b = synth.conv_input(cin=cout, cout=cout, T=T, H=H, W=W, seed=cout + 3)
+    pk = B.prepack_conv(w.cuda().bfloat16(), b.cuda())
+    y = B.causal_conv3d(to_cl(x), pk)
+    torch.cuda.synchronize()
+    yc = y.float().cpu()
+    seams = {(t, h, c) for t in (0, 3) for h in (0, 7, 8, 15, 16, 31, 32, 255)
+             for c in (0, 15, 16, 319)}
+    pts = sorted(set(sample_voxels(T, H, W, 512 - len(seams), seed=8)) | seams)
+    got = np.stack([yc[t, h, c].double().numpy() for (t, h, c) in pts], 1)
+    ref = np.stack([O.causal_conv3d_at(x, w, b, t, h, c) for (t, h, c) in pts], 1)
+    assert_close(got, ref, torch.bfloat16, f"conv {cout} many waves")
+    assert torch.isfinite(yc).all()
+    assert B.device_error() == 0

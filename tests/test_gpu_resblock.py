@@ -203,3 +203,19 @@ def test_trunk_cuda_graph_replay():
     g.z.copy_(zd2)
     assert torch.equal(g.replay().clone(), B.decode_trunk(zd2, tr))
     assert B.device_error() == 0
+
+
+def test_resblock_128_many_waves_sampled():
+    """Res block 128 -> 128 on [128, 4, 256, 320] (1,280 tiles per conv, conv1
+    with the fused norm2).  256 sampled voxels against the oracle."""
+    x, p = synth.resblock_input(cin=128, cout=128, T=4, H=256, W=320, seed=5)
+    blk = B.PackedResBlock(p)
+    y = B.resblock(to_cl(x), blk)
+    torch.cuda.synchronize()
+    yc = y.float().cpu()
+    seams = {(t, h, c) for t in (0, 3) for h in (0, 7, 8, 31, 32) for c in (0, 15, 16, 319)}
+    pts = sorted(set(sample_voxels(4, 256, 320, 256 - len(seams), seed=9)) | seams)
+    got = np.stack([yc[t, h, c].double().numpy() for (t, h, c) in pts], 1)
+    ref = np.stack([resblock_at(x, p, t, h, c) for (t, h, c) in pts], 1)
+    assert_close(got, ref, torch.bfloat16, "res block 128 many waves")
+    assert B.device_error() == 0
