@@ -1,6 +1,6 @@
 """The decoder trunk against the oracle where only large layers reach (GPU).
 
-Three kinds of comparison, all at the spec bf16 tolerances
+Three kinds of comparison, all at the bf16 path's tolerances
 (rel-L2 <= 1e-2, max |err| <= 5e-2 x std of the reference):
 
 * Every output element at sizes where the last stage runs more tiles than
