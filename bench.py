@@ -293,10 +293,14 @@ def oracle_sample_text(crop, spent, reps):
             f"{spent:.1f} s of oracle work")
 
 
-def bench_config(world):
+def bench_config(world, split="replicas"):
     """The `config` object of the JSON line (both arms print the same one)."""
+    if split == "rows":
+        par = f"one decode split by latent rows over {world} GPU(s), NCCL halo exchange"
+    else:
+        par = f"replicas x{world}" if world > 1 else "single GPU"
     return {"workload": WORKLOAD,
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "parallelism": par,
             "l2": "flushed before every timed step, outside the step events (512 MiB written, "
                   "then read back: no dirty line of the flush left)",
             "trunk_dense_tflop_per_step": sum(f for _, f in trunk_layers()) / 1e12}
@@ -536,6 +540,9 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--split", default="replicas", choices=["replicas", "rows"],
+                    help="replicas (default): one whole decode per GPU (weak scaling); rows: one "
+                         "decode split by latent rows over the GPUs (strong scaling)")
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", default=None,
@@ -575,8 +582,16 @@ def main():
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
 
+    rows = args.split == "rows"
+    if rows:
+        from video_diffusion_vae_b200 import shard
+        dec = shard.RowSplitDecoder(tr, T, H, W, rank, world, device=dev)
+
     def step():
-        B.decode_trunk(zd, tr, out=video, workspace=ws)
+        if rows:
+            dec.decode(zd)
+        else:
+            B.decode_trunk(zd, tr, out=video, workspace=ws)
 
     for _ in range(args.warmup):
         step()
@@ -600,7 +615,9 @@ def main():
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
     total_ms = sum(step_ms)
     max_total_ms = max_over_ranks(total_ms, dev)
-    value = throughput(T, args.steps, world, max_total_ms)
+    # replicas: every rank decodes; rows: the ranks decode one video together
+    job_decodes = 1 if rows else world
+    value = throughput(T, args.steps, job_decodes, max_total_ms)
     clocks = clk.summary()
 
     # ---- a second pass with events around every launch (the library records
@@ -665,19 +682,34 @@ def main():
                 vh[b].copy_(vdb[b], non_blocking=True)
                 d2h_done[b].record(d2h_s)
 
-    e2e_steps(3)
+    def e2e_rows(n):
+        # every rank copies the latents in; rank 0 copies the gathered video out
+        for _ in range(n):
+            zd.copy_(zh, non_blocking=True)
+            v = dec.decode(zd)
+            if v is not None:
+                vh[0].copy_(v, non_blocking=True)
+
+    run_e2e = e2e_rows if rows else e2e_steps
+    run_e2e(3)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_start.record(comp_s)
     h2d_s.wait_stream(comp_s)  # the first input copy starts inside the timed region
-    e2e_steps(args.steps)
+    run_e2e(args.steps)
     d2h_s.wait_stream(comp_s)
     t_end.record(d2h_s)
     torch.cuda.synchronize()
-    e2e_value = throughput(T, args.steps, world, max_over_ranks(t_start.elapsed_time(t_end), dev))
-    assert torch.equal(vh[(args.steps - 1) & 1].cuda(), video)  # the copied-out result is the decode
+    e2e_value = throughput(T, args.steps, job_decodes,
+                           max_over_ranks(t_start.elapsed_time(t_end), dev))
+    if rows:
+        # the gathered video is the whole decode's
+        if rank == 0:
+            assert torch.equal(vh[0].cuda(), B.decode_trunk(zd, tr))
+    else:
+        assert torch.equal(vh[(args.steps - 1) & 1].cuda(), video)  # the copied-out result is the decode
 
     err = B.device_error()
     comp = None
@@ -693,9 +725,9 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_total_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "scaling": "strong" if rows else "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) latents, random weights with the trunk's shapes)",
-            "config": bench_config(world),
+            "config": bench_config(world, args.split),
             "tflops": sum(f for _, f in layers) * args.steps / (total_ms * 1e-3) / 1e12,
             "roofline": {"bound": "tensor",
                          "kernel": "the 21 conv launches of a step: conv_tc_kernel x 20, head_tc_kernel x 1",

@@ -231,3 +231,79 @@ def test_row_slab_halo_plan():
     assert all(off + 2 * d[0] * d[1] * d[2] * d[3] <= ws for off, d in plan)
     off, dims = ctypes.c_size_t(0), (ctypes.c_int * 4)()
     assert lib.wvae_decode_rows_halo(22, 4, 11, 78, w, ctypes.byref(off), dims) == 1
+
+
+# ----------------------------------- the device driver's order, with gloo
+class _FakeSlab:
+    """Stands in for the library's row slab on the CPU: two launches that read
+    a halo (steps 1 and 2) and one that does not (step 0).  Each launch checks
+    that the halo rows of its input hold the neighbours' edge rows (or zeros
+    at the frame's edges) and then writes its own rows from them, so a missed
+    or misordered exchange changes the video."""
+
+    def __init__(self, T, rows, W, r0, H):
+        self.steps = 3
+        self.rows, self.r0, self.H = rows, r0, H
+        self.t = torch.zeros(T, rows + 2, W, 8, dtype=torch.bfloat16)
+        self.halo = [None, self.t, self.t]
+        self.ok = True
+
+    def step(self, i, z_rows, video_rows):
+        own = torch.arange(self.r0, self.r0 + self.rows, dtype=torch.float32)
+        if i == 0:      # the slab's own rows hold their global row index + 1
+            self.t[:, 1:-1] = (own + 1).view(1, -1, 1, 1).to(torch.bfloat16)
+            return
+        top = float(self.t[0, 0, 0, 0]); bot = float(self.t[0, -1, 0, 0])
+        self.ok &= top == (self.r0 if self.r0 > 0 else 0.0)
+        self.ok &= bot == (self.r0 + self.rows + 1 if self.r0 + self.rows < self.H else 0.0)
+        if i == 2:      # video rows: the row's value + its neighbours', 16 video rows a latent row
+            v = (self.t[:, :-2] + self.t[:, 1:-1] + self.t[:, 2:]).float()[..., 0]
+            video_rows[0, :, :, :, :] = v.repeat_interleave(16, 1)[:, :, :1].unsqueeze(0)
+
+
+def _driver_rank(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        T, H, W = 2, 5, 3
+        parts = shard.partition(H, world)
+        r0, r1 = parts[rank]
+        fake = _FakeSlab(T, r1 - r0, W, r0, H)
+        dec = shard.RowSplitDecoder(None, T, H, W, rank, world, device="cpu", slab=fake)
+        z = torch.zeros(1, 48, T, H, W, dtype=torch.bfloat16)
+        video = dec.decode(z)
+        ok = fake.ok
+        if rank == 0:
+            rows = torch.arange(1, H + 1, dtype=torch.float32)
+            pad = torch.cat([torch.zeros(1), rows, torch.zeros(1)])
+            want = (pad[:-2] + pad[1:-1] + pad[2:]).repeat_interleave(16)
+            ok = ok and video.shape == (1, 3, T, 16 * H, 16 * W) and \
+                torch.equal(video[0, 0, 0, :, 0].float(), want)
+        q.put((rank, bool(ok)))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_row_split_driver_exchanges_and_gathers(world):
+    """shard.RowSplitDecoder with gloo ranks: before every launch that reads
+    a halo, the halo rows hold the neighbours' edge rows (zeros at the
+    frame's edges); rank 0 receives every rank's video rows."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    ps = [ctx.Process(target=_driver_rank, args=(r, world, port, q)) for r in range(world)]
+    for p in ps:
+        p.start()
+    for p in ps:
+        p.join(120)
+    for p in ps:
+        if p.is_alive():
+            p.terminate()
+            p.join(10)
+    assert all(p.exitcode == 0 for p in ps), [p.exitcode for p in ps]
+    got = dict(q.get(timeout=10) for _ in range(world))
+    assert all(got.values()), got

@@ -139,6 +139,40 @@ def slab_latents(z: torch.Tensor, part: tuple[int, int]) -> torch.Tensor:
     return out.contiguous()
 
 
+class RowSplitDecoder:
+    """This rank's part of decodes split by latent rows over the ranks of
+    `group`: its row slab (workspace and halo views), its latents with their
+    halo rows and its video rows, set up once and reused by decode().
+    `slab` may be given (any object with the RowSlab interface: steps, halo,
+    step(i, z_rows, video_rows)); by default the library's row slab."""
+
+    def __init__(self, trunk, T: int, H: int, W: int, rank: int, world: int, group=None,
+                 device="cuda", slab=None):
+        self.rank, self.world, self.group = rank, world, group
+        self.parts = partition(H, world)
+        r0, r1 = self.parts[rank]
+        if slab is None:
+            from video_diffusion_vae_b200 import binding as B
+            slab = B.RowSlab(trunk, T, r1 - r0, W, device=device)
+        self.slab = slab
+        self.video = torch.empty((1, 3, T, 16 * (r1 - r0), 16 * W), dtype=torch.bfloat16,
+                                 device=device)
+
+    def decode(self, z, gather: bool = True):
+        """z: the whole latents [1, 48, T, H, W] (every rank passes the same).
+        Returns the whole video on rank 0 (gather=True; None elsewhere) or this
+        rank's video rows."""
+        zr = slab_latents(z, self.parts[self.rank])
+        sl = self.slab
+        for i in range(sl.steps):
+            if sl.halo[i] is not None:
+                exchange_halo(sl.halo[i], self.rank, self.world, 1, self.group)
+            sl.step(i, zr, self.video)
+        if not gather:
+            return self.video
+        return gather_rows(self.video, self.parts, 16, self.rank, self.world, 3, self.group)
+
+
 def decode_rows(z, trunk, rank: int, world: int, group=None, gather: bool = True):
     """One decode split over the ranks of `group` by latent rows (every rank
     passes the same latents z [1, 48, T, H, W], bf16, on its GPU).  Each rank
@@ -146,20 +180,9 @@ def decode_rows(z, trunk, rank: int, world: int, group=None, gather: bool = True
     halo rows of every 3x3 conv's input with its neighbours (NCCL point-to-
     point for CUDA tensors).  Returns the whole video on rank 0 (gather=True,
     as the pages' decoder does) or this rank's video rows."""
-    from video_diffusion_vae_b200 import binding as B
     _, _, T, H, W = z.shape
-    parts = partition(H, world)
-    r0, r1 = parts[rank]
-    slab = B.RowSlab(trunk, T, r1 - r0, W, device=z.device)
-    zr = slab_latents(z, (r0, r1))
-    video = torch.empty((1, 3, T, 16 * (r1 - r0), 16 * W), dtype=torch.bfloat16, device=z.device)
-    for i in range(slab.steps):
-        if slab.halo[i] is not None:
-            exchange_halo(slab.halo[i], rank, world, 1, group)
-        slab.step(i, zr, video)
-    if not gather:
-        return video
-    return gather_rows(video, parts, 16, rank, world, 3, group)
+    dec = RowSplitDecoder(trunk, T, H, W, rank, world, group, device=z.device)
+    return dec.decode(z, gather)
 
 
 def decode_rows_emulated(z, trunk, world: int):
