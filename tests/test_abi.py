@@ -187,3 +187,28 @@ def test_video_decode_frames_and_validation():
     assert lib.wvae_decode_video(P, N, A, A, 4, H, W, w, B.BF16, A, ws, NULL, 0, 1, NULL) == 1
     assert lib.wvae_decode_video(P, N, A, A, 1, H, W, w, B.BF16, A, ws, A, 1 << 40, 0, NULL) == 1
     assert lib.wvae_decode_video(P, N, A, A, 4, H, W, w, B.BF16, A, 1024, NULL, 0, 0, NULL) == 4
+
+
+def test_winograd_and_row_slab_entry_points_reject_on_host():
+    """Refused before any launch: Winograd conv with input channels not a
+    multiple of 64, an unsupported output width, aliasing; row-slab steps out
+    of range and a slab whose last stage is wider than the head kernel takes."""
+    lib = B.load()
+    assert lib.wvae_conv_winograd_packed_bytes(64, 64) > lib.wvae_conv_packed_bytes(64, 64, 3, 3, 3, 0)
+    ws = lib.wvae_causal_conv3d_winograd_workspace_bytes(2, 9, 17, 64, 64)
+    assert ws == 2 * (-(-16 * 2 * 5 * 9 * 64 * 2 // 256) * 256)
+    A2 = ctypes.c_void_p(0x20000)
+    assert lib.wvae_causal_conv3d_winograd(A, A2, 2, 9, 17, 32, 64, NULL, A2, A, ws, NULL) in (1, 2, 3)
+    assert lib.wvae_causal_conv3d_winograd(A, A2, 2, 9, 17, 64, 72, NULL, A2, A, ws, NULL) in (2, 3)
+    assert lib.wvae_causal_conv3d_winograd(A, A2, 2, 9, 17, 64, 64, NULL, A, A, ws, NULL) == 1
+    w = (ctypes.c_int * 4)(128, 128, 64, 64)
+    P = (ctypes.c_void_p * 21)(*([A] * 21))
+    N = (ctypes.c_void_p * 34)(*([A] * 34))
+    assert lib.wvae_decode_rows_step(22, P, N, A, A, 2, 3, 4, w, B.BF16, A, 1 << 40, NULL) == 1
+    assert lib.wvae_decode_rows_step(-1, P, N, A, A, 2, 3, 4, w, B.BF16, A, 1 << 40, NULL) == 1
+    off, dims = ctypes.c_size_t(0), (ctypes.c_int * 4)()
+    wide = (ctypes.c_int * 4)(128, 128, 64, 256)
+    # a last stage wider than the head kernel takes: the whole slab plan is refused
+    assert lib.wvae_decode_rows_halo(3, 2, 3, 4, wide, ctypes.byref(off), dims) == 2
+    assert lib.wvae_decode_rows_halo(21, 2, 3, 4, wide, ctypes.byref(off), dims) == 2
+    assert lib.wvae_decode_rows_halo(3, 2, 3, 4, w, ctypes.byref(off), dims) == 0

@@ -46,3 +46,19 @@ def test_row_split_full_size_equals_whole(world):
     assert video.shape == whole.shape == (1, 3, 4, 704, 1248)
     assert torch.equal(video, whole), (video.float() - whole.float()).abs().max().item()
     assert B.device_error() == 0
+
+
+def test_row_split_one_row_slabs():
+    """Three latent rows over three slabs: every slab holds one own row between
+    two halo rows at stage 0 (and 8 at stage 3); the assembled video equals the
+    whole decode and the oracle."""
+    z, params = synth.trunk_input(T=2, H=3, W=4, widths=(128, 128, 64, 64), seed=43)
+    tr = B.PackedTrunk(params)
+    zd = z[None].cuda().bfloat16().contiguous()
+    video = shard.decode_rows_emulated(zd, tr, 3)
+    whole = B.decode_trunk(zd, tr)
+    torch.cuda.synchronize()
+    assert torch.equal(video, whole)
+    assert_close(video[0].float().cpu().double().numpy(), O.trunk(z, params), torch.bfloat16,
+                 "one-row slabs")
+    assert B.device_error() == 0

@@ -182,3 +182,21 @@ def test_video_decode_full_size_properties():
     assert torch.equal(v[:, :, :9], v2[:, :, :9])
     assert not torch.equal(v[:, :, 9], v2[:, :, 9])
     assert B.device_error() == 0
+
+
+# ------------------------------------------------------------- edge cases
+def test_trunk_and_video_single_latent_frame():
+    """T = 1: every causal conv sees only its current frame (two zero frames in
+    front), and the video decode with temporal upsampling keeps the single
+    frame once (4T - 3 = 1): both equal the oracle's trunk."""
+    z, params = synth.trunk_input(T=1, H=3, W=5, widths=(128, 128, 64, 64), seed=41)
+    tr = B.PackedTrunk(params)
+    zd = z[None].cuda().bfloat16().contiguous()
+    v = B.decode_trunk(zd, tr)
+    vv = B.decode_video(zd, tr)
+    torch.cuda.synchronize()
+    assert v.shape == vv.shape == (1, 3, 1, 48, 80)
+    ref = O.trunk(z, params)
+    assert_close(v[0].float().cpu().double().numpy(), ref, torch.bfloat16, "trunk T=1")
+    assert_close(vv[0].float().cpu().double().numpy(), ref, torch.bfloat16, "video T=1")
+    assert B.device_error() == 0
