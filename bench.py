@@ -446,6 +446,31 @@ def components(peaks, flush, reps=10):
     out["conv_256x256_4x176x312_winograd"] = {"ms": mw, "TFLOP/s_dense_equiv": fl / mw / 1e9,
                                                "vs_direct": md / mw}
     del xd, y, pk, pw, wsw
+    # the pages' video length: latents [1,48,49,44,78] -> 193 frames of 704 x 1248,
+    # decoded in streaming chunks of 5 + 11 x 4 latent frames (temporal 2x steps,
+    # causal caches carried between chunks)
+    z49, p49 = synth.trunk_input(T=49, H=44, W=78, seed=2)
+    tr49 = B.PackedTrunk(p49)
+    zd49 = z49[None].cuda().bfloat16().contiguous()
+    bounds = [0, 5] + [5 + 4 * k for k in range(1, 12)]
+    zchunks = [zd49[:, :, a:b].contiguous() for a, b in zip(bounds, bounds[1:])]
+    outs = [torch.empty((1, 3, B.video_frames(b - a, i > 0), 704, 1248), dtype=torch.bfloat16,
+                        device="cuda") for i, (a, b) in enumerate(zip(bounds, bounds[1:]))]
+    vs = B.VideoStream(tr49, 44, 78)
+    wsv = torch.empty(tr49.video_workspace_bytes(5, 44, 78), dtype=torch.uint8, device="cuda")
+
+    def decode_193():
+        vs.started = False
+        for zc, oc in zip(zchunks, outs):
+            vs.decode(zc, out=oc, workspace=wsv)
+    med, _ = time_events(decode_193, 3, 1, flush)
+    nfr = sum(o.shape[2] for o in outs)
+    assert nfr == 193
+    out["video_193_frames_chunked"] = {
+        "ms": med, "frames/s": nfr / (med * 1e-3),
+        "workload": "latents [1,48,49,44,78] -> video [1,3,193,704,1248] (the trunk with its "
+                    "temporal 2x steps), chunks of 5 + 11 x 4 latent frames"}
+    del zd49, zchunks, outs, vs, wsv, tr49
     for cout in (256, 128):
         x, p = synth.resblock_input(cout=cout)
         blk = B.PackedResBlock(p)
