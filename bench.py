@@ -8,12 +8,17 @@ norm_out + SiLU + head conv + pixel shuffle.  It runs every step of the hot
 path; value = decoded frames/s over all ranks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--split replicas|rows]
 
-Under torchrun each rank decodes its own replica (the trunk has no exchange
-step: "replicas only"); the timed region is bracketed by a barrier and a
-device synchronise and its duration is the max over ranks.  `--impl
-reference` times the CPU oracle instead (rank 0 only), on a bounded sample.
-Rank 0 prints one JSON line.
+Under torchrun each rank decodes its own replica by default (weak scaling);
+with `--split rows` the ranks decode one video together, split by latent
+rows with the halo rows exchanged over NCCL (strong scaling).  The timed
+region is bracketed by a barrier and a device synchronise and its duration
+is the max over ranks.  Besides the trunk the line carries the components:
+norm-SiLU, the causal conv (direct and Winograd), the residual block, and
+the 193-frame video of 49 latent frames streamed with temporal upsampling.
+`--impl reference` times the CPU oracle instead (rank 0 only), one bounded
+layer-shape sample per step.  Rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
