@@ -219,3 +219,22 @@ def test_resblock_128_many_waves_sampled():
     ref = np.stack([resblock_at(x, p, t, h, c) for (t, h, c) in pts], 1)
     assert_close(got, ref, torch.bfloat16, "res block 128 many waves")
     assert B.device_error() == 0
+
+
+def test_trunk_timed_decode_equals_plain_and_records_every_launch():
+    """wvae_decode_trunk_timed (the benchmark's per-launch timing) enqueues the
+    same work as wvae_decode_trunk: the same video bit for bit, and an event
+    pair around each of the 22 launches (the event clock ticks every ~2 us, so
+    a small launch may read 0; the total is positive)."""
+    z, params = synth.trunk_input(T=2, H=3, W=5, widths=(128, 128, 64, 64), seed=6)
+    tr = B.PackedTrunk(params)
+    zd = z[None].cuda().bfloat16().contiguous()
+    plain = B.decode_trunk(zd, tr)
+    n = B.trunk_launches()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n)]
+    timed = B.decode_trunk(zd, tr, events=ev)
+    torch.cuda.synchronize()
+    assert torch.equal(plain, timed)
+    durations = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(n)]
+    assert n == 22 and all(d >= 0 for d in durations) and sum(durations) > 0
+    assert B.device_error() == 0
