@@ -53,9 +53,9 @@ def test_trunk_multi_tile_vs_oracle(widths):
     assert B.device_error() == 0
 
 
-def _read_golden():
+def _read_golden(path=GOLDEN):
     meta, rows = {}, []
-    with open(GOLDEN) as f:
+    with open(path) as f:
         for line in f:
             if line.startswith("#"):
                 continue
@@ -199,4 +199,37 @@ def test_trunk_and_video_single_latent_frame():
     ref = O.trunk(z, params)
     assert_close(v[0].float().cpu().double().numpy(), ref, torch.bfloat16, "trunk T=1")
     assert_close(vv[0].float().cpu().double().numpy(), ref, torch.bfloat16, "video T=1")
+    assert B.device_error() == 0
+
+
+VIDEO_GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                            "trunk_video_full_size_samples.txt")
+
+
+def test_video_decode_full_size_vs_oracle_samples():
+    """The 4T - 3 decode at full size: latents [1, 48, 4, 44, 78] (seed 0) ->
+    video [1, 3, 13, 704, 1248], at ~10,000 pixels (every channel on frames
+    0, 1, 2, 5, 9, 12 at the crossings of 18 rows and 16 columns on tile
+    seams and frame edges, plus 5,000 uniform) against oracle values stored
+    by tests/golden/make_trunk_full_size_samples.py --video; the max-error
+    bound uses the std of the whole oracle video.  Covers the temporal 2x
+    steps written by the upsample convs' epilogues at full size (stages 1-3
+    on 7 and 13 frames, several tiles per CTA everywhere)."""
+    meta, rows = _read_golden(VIDEO_GOLDEN)
+    z, params = synth.trunk_input(T=4, H=44, W=78, seed=0)
+    tr = B.PackedTrunk(params)
+    video = B.decode_video(z[None].cuda().bfloat16().contiguous(), tr)
+    torch.cuda.synchronize()
+    assert video.shape == (1, 3, 13, 704, 1248)
+    v = video[0].float().cpu()
+    idx = torch.tensor([r[:4] for r in rows])
+    got = v[idx[:, 0], idx[:, 1], idx[:, 2], idx[:, 3]].double().numpy()
+    ref = np.array([r[4] for r in rows])
+    assert np.isfinite(got).all()
+    d = got - ref
+    rel = np.linalg.norm(d) / np.linalg.norm(ref)
+    mx = np.abs(d).max() / meta["std"]
+    assert rel <= REL_L2_BF16, f"rel L2 {rel:.3e}"
+    assert mx <= MAX_ABS_BF16, f"max |err| / std {mx:.3e}"
+    assert abs(v.double().std().item() / meta["std"] - 1.0) < 1e-2
     assert B.device_error() == 0
