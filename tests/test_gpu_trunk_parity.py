@@ -233,3 +233,27 @@ def test_video_decode_full_size_vs_oracle_samples():
     assert mx <= MAX_ABS_BF16, f"max |err| / std {mx:.3e}"
     assert abs(v.double().std().item() / meta["std"] - 1.0) < 1e-2
     assert B.device_error() == 0
+
+
+def test_video_decode_193_frames_whole_equals_streamed():
+    """The pages' video length in one call: latents [1, 48, 49, 44, 78] ->
+    video [1, 3, 193, 704, 1248].  The whole decode's stage-3 tensors hold
+    5.4 G elements (offsets past 2^31; ~50 GB of workspace); the streamed
+    decode (chunks of 5 + 11 x 4 latent frames) never more than 0.6 G.  Each
+    chunk's video equals its frames of the whole decode bit for bit."""
+    z, params = synth.trunk_input(T=49, H=44, W=78, seed=5)
+    tr = B.PackedTrunk(params)
+    zd = z[None].cuda().bfloat16().contiguous()
+    whole = B.decode_video(zd, tr)
+    assert whole.shape == (1, 3, 193, 704, 1248)
+    stream = B.VideoStream(tr, 44, 78)
+    t0 = 0
+    for n in [5] + [4] * 11:
+        part = stream.decode(zd[:, :, t0:t0 + n].contiguous())
+        f0 = 0 if t0 == 0 else 4 * t0 - 3
+        assert part.shape[2] == (4 * n - 3 if t0 == 0 else 4 * n)
+        assert torch.equal(part, whole[:, :, f0:f0 + part.shape[2]]), f"chunk at latent frame {t0}"
+        t0 += n
+    assert t0 == 49
+    assert torch.isfinite(whole).all()
+    assert B.device_error() == 0
