@@ -226,6 +226,13 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   const bool kwn = p.BN == 16 && a.KH == 3 && a.KW == 3 && a.phases == 1 && a.cin2_pad == 0 &&
                    a.ep.act == nullptr && a.ep.residual == nullptr && p.nsplit == 1;
   p.nw = kwn ? a.KW : 1;
+  // CTA pairs (M = 256 MMAs, each CTA loading half of every weight tile) for
+  // the 128- and 256-wide N tiles of direct convs: half the weight bytes per
+  // SM through the fill and shared memory.
+  p.pair = (p.nsplit == 1 && (p.BN == 128 || p.BN == 256) && p.nw == 1 && !a.wino &&
+            a.cin2_pad == 0)
+               ? 1
+               : 0;
   p.num_acc = 2 * p.S * static_cast<int>(conv_tc_acc_stride(p)) <= 512 ? 2 : 1;
   // Row taps share one A window (the tile plus its row halo) per (kt, kw); up
   // to 128 output channels a B stage carries all of a window's row taps.
@@ -272,7 +279,7 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   auto a32 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 31u) == 0; };
   p.ep.vec32 = (a.cout % 16 == 0 && a32(a.ep.residual) && a32(a.ep.out) && a32(a.ep.act)) ? 1 : 0;
   p.err = d.err;
-  const int box_rows = p.BN;  // BN <= 256
+  const int box_rows = conv_tc_b_rows(p);  // BN <= 256, or BN / 2 with a pair
   const int a_rows = static_cast<int>(conv_tc_a_rows(p));
   if (a.wino) {
     if (!encode_planes(&p.tmA, a.x, a.cin_pad, a.W, a.H, a.T, p.tile_cols, a_rows))
@@ -298,10 +305,12 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
                         ? 1
                         : 0;
   int grid;
-  if (p.nsplit == 2) {
+  if (p.nsplit == 2 || p.pair) {
     int clusters = conv_tc_max_clusters(p);
     if (clusters < 1) clusters = d.num_sms / 2;
-    grid = 2 * (p.num_tiles < clusters ? p.num_tiles : clusters);
+    // a pair takes two spatial tiles of one (N tile, phase) at a time
+    const int units = p.pair ? ((p.m_tiles + 1) / 2) * p.phases * p.n_tiles : p.num_tiles;
+    grid = 2 * (units < clusters ? units : clusters);
   } else {
     grid = p.num_tiles < d.num_sms ? p.num_tiles : d.num_sms;
   }

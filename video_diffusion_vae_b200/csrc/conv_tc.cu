@@ -112,7 +112,11 @@ struct TileCoord {
 // frames read the same input frames: a frame of a large layer does not stay
 // in L2 until the next frame's tiles come round), then tile column and row.
 // With nsplit = 2 the two CTAs of a cluster take the same tiles and the CTA
-// rank is the N tile.
+// rank is the N tile.  With a pair, loop index t names an (N tile, phase) and
+// a pair of spatial M tiles: rank r takes spatial tile 2i + r (both CTAs of a
+// pair multiply by the same weights); when the count of spatial tiles is odd
+// the last pair's rank 1 takes a copy of the last one so that the pair's MMAs
+// stay whole, and writes nothing (tile_own).
 __device__ __forceinline__ TileCoord decode_tile(const ConvParams& p, int tile, int crank) {
   TileCoord c;
   int m;
@@ -125,6 +129,10 @@ __device__ __forceinline__ TileCoord decode_tile(const ConvParams& p, int tile, 
   }
   c.phase = m % p.phases;
   m /= p.phases;
+  if (p.pair) {
+    m = 2 * m + crank;
+    if (m >= p.m_tiles) m = p.m_tiles - 1;
+  }
   c.t = m % p.T;
   m /= p.T;
   c.tw = m % p.tiles_w;
@@ -133,11 +141,21 @@ __device__ __forceinline__ TileCoord decode_tile(const ConvParams& p, int tile, 
 }
 
 // ------------------------------------------------------------------ producer
+// Every role walks the same sequence of loop indices: tile_first, then steps
+// of tile_stride, below tile_count; the two CTAs of a cluster (nsplit = 2 or
+// a pair) share each index (decode_tile).
+__device__ __forceinline__ bool cluster2(const ConvParams& p) { return p.nsplit == 2 || p.pair; }
 __device__ __forceinline__ int tile_first(const ConvParams& p) {
-  return p.nsplit == 2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  return cluster2(p) ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
 }
 __device__ __forceinline__ int tile_stride(const ConvParams& p) {
-  return p.nsplit == 2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  return cluster2(p) ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+}
+__device__ __forceinline__ int tile_count(const ConvParams& p) {
+  return p.pair ? ((p.m_tiles + 1) >> 1) * p.phases * p.n_tiles : p.num_tiles;
+}
+__device__ __forceinline__ bool tile_own(const ConvParams& p, int t, int crank) {
+  return !p.pair || 2 * (t / (p.n_tiles * p.phases)) + crank < p.m_tiles;
 }
 
 // Waits, bounded, until every copy this thread issued into a ring has landed.
@@ -155,15 +173,34 @@ __device__ void drain_ring(const uint64_t* full, uint32_t issued, int stages, un
 // tiles of taps (kt, 0..kh_eff-1, kw) to the B ring, b_tiles per stage.  A
 // second-segment group (1x1x1 shortcut) is one A tile without halo and one
 // weight tile (alone in its B stage).
+template <bool PAIR>
 __device__ void producer(const ConvParams& p, const Smem& s, int crank) {
   const int cchunks = p.cin_pad / kBK;
   const uint32_t a_tx_main = conv_tc_a_rows(p) * static_cast<uint32_t>(p.tile_cols) * 128u;
   const uint32_t a_tx_sc = static_cast<uint32_t>(p.tile_rows * p.tile_cols) * 128u;
-  const uint32_t tile_tx = static_cast<uint32_t>(p.BN) * 128u;
+  const uint32_t tile_tx = static_cast<uint32_t>(conv_tc_b_rows(p)) * 128u;
   const int kw_stride = p.kw_eff * p.nw;  // tap = ((kt kh_eff + kh) kw_stride + kw) (+ phase)
+  // With a pair each CTA loads its own A window and half of each weight tile;
+  // both halves complete on rank 0's barrier, which rank 0 alone arms for the
+  // bytes of both CTAs.
+  const int b_row0 = PAIR ? crank * conv_tc_b_rows(p) : 0;
+  const bool arms = !PAIR || crank == 0;
+  const uint32_t tx_mul = PAIR ? 2u : 1u;
+  auto bar_of = [&](const uint64_t* b) {
+    if constexpr (PAIR)
+      return mapa_shared(smem_u32(b), 0);
+    else
+      return smem_u32(b);
+  };
+  auto load4 = [&](uint32_t dst, const CUtensorMap* m, uint32_t bar, int c0, int c1, int c2, int c3) {
+    if constexpr (PAIR)
+      tma_load_4d_pair(dst, m, bar, c0, c1, c2, c3);
+    else
+      tma_load_4d(dst, m, bar, c0, c1, c2, c3);
+  };
   uint32_t ia = 0, ib = 0;
   bool aborted = false;
-  for (int tile = tile_first(p); tile < p.num_tiles && !aborted; tile += tile_stride(p)) {
+  for (int tile = tile_first(p); tile < tile_count(p) && !aborted; tile += tile_stride(p)) {
     const TileCoord tc = decode_tile(p, tile, crank);
     const int h0 = tc.th * p.tile_rows, w0 = tc.tw * p.out_cols;
     // output (h, w) reads input row h + oh + kh and column w + ow + kw; phase
@@ -191,11 +228,11 @@ __device__ void producer(const ConvParams& p, const Smem& s, int crank) {
           if (p.wino)
             tma_load_5d(dst, &p.tmA, bar, cc * kBK, w0, h0, ts, tc.phase);
           else if (ts < 0 && p.has_cache)
-            tma_load_4d(dst, &p.tmC, bar, cc * kBK, w0 + ow + kw, h0 + oh, ts + p.KT - 1);
+            load4(dst, &p.tmC, bar, cc * kBK, w0 + ow + kw, h0 + oh, ts + p.KT - 1);
           else
-            tma_load_4d(dst, &p.tmA, bar, cc * kBK, w0 + ow + kw, h0 + oh, ts);
+            load4(dst, &p.tmA, bar, cc * kBK, w0 + ow + kw, h0 + oh, ts);
         } else {
-          tma_load_4d(dst, &p.tmA2, bar, cc * kBK, w0, h0, tc.t);
+          load4(dst, &p.tmA2, bar, cc * kBK, w0, h0, tc.t);
         }
       };
       if (!p.combined) {
@@ -205,8 +242,8 @@ __device__ void producer(const ConvParams& p, const Smem& s, int crank) {
           aborted = true;
           break;
         }
-        const uint32_t bar = smem_u32(&s.full_a[st]);
-        mbar_arrive_expect_tx(bar, a_tx);
+        const uint32_t bar = bar_of(&s.full_a[st]);
+        if (arms) mbar_arrive_expect_tx(smem_u32(&s.full_a[st]), tx_mul * a_tx);
         load_a(smem_u32(s.a_ring + st * s.a_bytes), bar);
         ++ia;
       }
@@ -219,32 +256,42 @@ __device__ void producer(const ConvParams& p, const Smem& s, int crank) {
           aborted = true;
           break;
         }
-        const uint32_t bar = smem_u32(&s.full_b[st]);
+        const uint32_t bar = bar_of(&s.full_b[st]);
         const uint32_t dst = smem_u32(s.b_ring + st * s.b_bytes);
         const uint32_t b_tx = main_seg ? s.b_bytes : tile_tx;
         if (p.combined) {
           // one stage per group: A slot st travels with B slot st on one barrier
-          mbar_arrive_expect_tx(bar, a_tx + b_tx);
+          if (arms) mbar_arrive_expect_tx(smem_u32(&s.full_b[st]), tx_mul * (a_tx + b_tx));
           load_a(smem_u32(s.a_ring + st * s.a_bytes), bar);
-        } else {
-          mbar_arrive_expect_tx(bar, b_tx);
+        } else if (arms) {
+          mbar_arrive_expect_tx(smem_u32(&s.full_b[st]), tx_mul * b_tx);
         }
+        auto load_b = [&](uint32_t d, const CUtensorMap* m, int c0, int c1) {
+          if constexpr (PAIR)
+            tma_load_2d_pair(d, m, bar, c0, c1);
+          else
+            tma_load_2d(d, m, bar, c0, c1);
+        };
         if (main_seg) {
-          // weight tiles [row tap j][column tap u], BN rows each
+          // weight tiles [row tap j][column tap u], BN rows each (BN / 2 with a pair)
           for (int j = 0; j < per_stage; ++j)
             for (int u = 0; u < p.nw; ++u) {
               const int tap = tap0 + (kt * p.kh_eff + kh0 + j) * kw_stride + kw + u;
-              tma_load_2d(dst + (j * p.nw + u) * tile_tx, &p.tmB, bar,
-                          tap * p.cin_pad + cc * kBK, tc.n_tile * p.BN);
+              load_b(dst + (j * p.nw + u) * tile_tx, &p.tmB, tap * p.cin_pad + cc * kBK,
+                     tc.n_tile * p.BN + b_row0);
             }
         } else {
-          tma_load_2d(dst, &p.tmB2, bar, cc * kBK, tc.n_tile * p.BN);
+          load_b(dst, &p.tmB2, cc * kBK, tc.n_tile * p.BN + b_row0);
         }
       }
       if (aborted) break;
     }
   }
-  // Do not leave while copies issued by this thread may still be landing.
+  // Do not leave while copies issued by this thread may still be landing.  A
+  // pair's rank 1 has no barriers of its own for them: rank 0 drains the
+  // shared ones, and neither CTA leaves before the other (the kernel's last
+  // cluster barrier).
+  if (PAIR && crank != 0) return;
   drain_ring(s.full_a, ia, p.stages_a, p.err);
   drain_ring(s.full_b, ib, p.stages_b, p.err);
 }
@@ -267,27 +314,43 @@ __device__ __forceinline__ bool mma_wait(uint32_t bar, uint32_t ph, const Smem& 
 }
 
 // COMBINED: a group's A window and weight tiles share one stage and barrier.
-template <int S, int KHT, int BT, bool COMBINED>
+// PAIR: M = 256 MMAs over the CTA pair (issued by rank 0 only), commits
+// multicast to the barriers of both CTAs.
+template <int S, int KHT, int BT, bool COMBINED, bool PAIR>
 __device__ void mma_issuer(const ConvParams& p, const Smem& s, uint32_t tmem_base) {
   static_assert(BT == 1 || BT == KHT, "a B stage holds one weight tile or the group's row taps");
   static_assert(!COMBINED || BT == KHT, "a combined stage holds all of a group's weight tiles");
   const uint32_t n_mma = static_cast<uint32_t>(p.nw * p.BN);  // N of one MMA
-  const uint32_t idesc = p.wino ? umma_idesc_f16(kBM, static_cast<int>(n_mma))
-                                : umma_idesc_bf16(kBM, static_cast<int>(n_mma));
+  const int m_mma = PAIR ? 2 * kBM : kBM;
+  const uint32_t idesc = p.wino ? umma_idesc_f16(m_mma, static_cast<int>(n_mma))
+                                : umma_idesc_bf16(m_mma, static_cast<int>(n_mma));
+  auto mma = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t acc) {
+    if constexpr (PAIR)
+      umma_bf16_pair(d, a, b, idesc, acc);
+    else
+      umma_bf16(d, a, b, idesc, acc);
+  };
+  auto commit = [&](uint32_t bar) {
+    if constexpr (PAIR)
+      umma_commit_pair_both(bar);
+    else
+      umma_commit(bar);
+  };
   // Descriptors of stage 0 of each ring; the start field counts 16-byte units.
   const uint64_t adesc0 = umma_desc_sw128(smem_u32(s.a_ring));
   const uint64_t bdesc0 = umma_desc_sw128(smem_u32(s.b_ring));
   const uint32_t a_step = s.a_bytes >> 4, b_step = s.b_bytes >> 4;
   const uint32_t sub_step = (static_cast<uint32_t>(kBM) * 128u) >> 4;
   const uint32_t kh_step = static_cast<uint32_t>(p.tile_cols) * 8u;  // tile_cols * 128 B / 16
-  const uint32_t tap_step = n_mma * 8u;  // one row tap's weight tiles: nw BN * 128 B / 16
+  // one row tap's weight tiles in the B stage: nw x (BN, or BN / 2 with a pair) rows x 128 B / 16
+  const uint32_t tap_step = static_cast<uint32_t>(p.nw * conv_tc_b_rows(p)) * 8u;
   const uint32_t full_a0 = smem_u32(&s.full_a[0]), empty_a0 = smem_u32(&s.empty_a[0]);
   const uint32_t full_b0 = smem_u32(&s.full_b[0]), empty_b0 = smem_u32(&s.empty_b[0]);
   const uint32_t n_stride = conv_tc_acc_stride(p);  // TMEM columns per sub-tile
   const uint32_t acc_cols = static_cast<uint32_t>(S) * n_stride;
   uint32_t sa = 0, pa = 0, sb = 0, pb = 0, ai = 0;
   bool aborted = false;
-  for (int tile = tile_first(p); tile < p.num_tiles && !aborted; tile += tile_stride(p), ++ai) {
+  for (int tile = tile_first(p); tile < tile_count(p) && !aborted; tile += tile_stride(p), ++ai) {
     const uint32_t acc = ai % p.num_acc;
     const uint32_t aph = (ai / p.num_acc) & 1u;
     if (!mbar_wait_bounded(smem_u32(&s.tempty[acc]), aph ^ 1u, s.abort_flag, p.err,
@@ -313,12 +376,12 @@ __device__ void mma_issuer(const ConvParams& p, const Smem& s, uint32_t tmem_bas
           const uint32_t accumulate = (k | kh) != 0 ? 1u : first;
 #pragma unroll
           for (int sub = 0; sub < S; ++sub)
-            umma_bf16(d_tmem + static_cast<uint32_t>(sub) * n_stride, a_kh + sub * sub_step + 2u * k,
-                      b_st + 2u * k, idesc, accumulate);
+            mma(d_tmem + static_cast<uint32_t>(sub) * n_stride, a_kh + sub * sub_step + 2u * k,
+                b_st + 2u * k, accumulate);
         }
       };
       auto release_b = [&]() {
-        umma_commit(empty_b0 + sb * 8u);
+        commit(empty_b0 + sb * 8u);
         if (++sb == static_cast<uint32_t>(p.stages_b)) {
           sb = 0;
           pb ^= 1u;
@@ -349,7 +412,7 @@ __device__ void mma_issuer(const ConvParams& p, const Smem& s, uint32_t tmem_bas
       }
       if (aborted) break;
       if (!COMBINED) {
-        umma_commit(empty_a0 + sa * 8u);
+        commit(empty_a0 + sa * 8u);
         if (++sa == static_cast<uint32_t>(p.stages_a)) {
           sa = 0;
           pa ^= 1u;
@@ -357,10 +420,13 @@ __device__ void mma_issuer(const ConvParams& p, const Smem& s, uint32_t tmem_bas
       }
     }
     if (aborted) break;
-    umma_commit(smem_u32(&s.tfull[acc]));
+    commit(smem_u32(&s.tfull[acc]));
   }
   // Every MMA issued by this thread has finished before TMEM/smem go away.
-  umma_commit(smem_u32(s.drain));
+  if constexpr (PAIR)
+    umma_commit_pair_local(smem_u32(s.drain));
+  else
+    umma_commit(smem_u32(s.drain));
   volatile int never = 0;
   mbar_wait_bounded(smem_u32(s.drain), 0, &never, p.err, DEVERR_TIMEOUT_DRAIN, kDrainLimitNs);
 }
@@ -757,6 +823,7 @@ __device__ __noinline__ void lane_emit_taps_in_n(const ConvParams& p, const Smem
   if (valid) emit_chunk<NB>(p, 0, n0, tc, h, w, vox, v);
 }
 
+template <bool PAIR>
 __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base, int warp,
                          int lane, int crank) {
   const int q = warp & 3;           // TMEM lane quarter this warp may access
@@ -769,7 +836,16 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
   // accumulator fills TMEM and CTAs run several tiles).
   const bool early = p.early_release != 0;
   uint32_t ti = 0;
-  for (int tile = tile_first(p); tile < p.num_tiles; tile += tile_stride(p), ++ti) {
+  // The accumulator's release: on this CTA's barrier, or on rank 0's with a
+  // pair (rank 0's MMAs write both CTAs' accumulators).
+  auto release = [&](uint32_t acc) {
+    tc_fence_before();
+    if constexpr (PAIR)
+      mbar_arrive_cluster(mapa_shared(smem_u32(&s.tempty[acc]), 0));
+    else
+      mbar_arrive(smem_u32(&s.tempty[acc]));
+  };
+  for (int tile = tile_first(p); tile < tile_count(p); tile += tile_stride(p), ++ti) {
     const uint32_t acc = ti % p.num_acc;
     const uint32_t aph = (ti / p.num_acc) & 1u;
     int ok = 0;
@@ -783,6 +859,7 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
     __syncwarp();  // order the other lanes' reads after lane 0's acquire
     tc_fence_after();
     const TileCoord tc = decode_tile(p, tile, crank);
+    const bool own = tile_own(p, tile, crank);
     const int n0 = tc.n_tile * p.BN;
     for (int sub = grp; sub < p.S; sub += 2) {  // the groups take alternate sub-tiles
       const int idx = sub * kBM + row;  // computed voxel of the tile, row-major
@@ -793,7 +870,7 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
       // 2h + p' - out_row0 of an out_rows-row output, or nowhere
       const int ho = p.phases == 4 ? 2 * h + (tc.phase >> 1) - p.out_row0 : h;
       const int Ho = p.out_rows > 0 ? p.out_rows : 2 * p.H;
-      const bool valid = h < p.H && w < p.W && (p.nw == 1 || (c >= 1 && c <= p.tile_cols - 2)) &&
+      const bool valid = own && h < p.H && w < p.W && (p.nw == 1 || (c >= 1 && c <= p.tile_cols - 2)) &&
                          (p.out_rows == 0 || (ho >= 0 && ho < p.out_rows));
       // output voxel: (t, h, w), or (t, 2h + p', 2w + q') of the 2H x 2W output in phase
       // mode.  With a temporal 2x step (phase mode only) input frame t goes to output
@@ -824,10 +901,7 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
         lane_emit(p, s, taddr, 0, p.BN, n0, valid, vox, vox2, tc, h, w);
       } else {
         float ss = lane_pass1(p, s, taddr, 0, p.BN, n0, valid, vox, vox2, !early);
-        if (early) {
-          tc_fence_before();
-          mbar_arrive(smem_u32(&s.tempty[acc]));
-        }
+        if (early) release(acc);
         if (p.nsplit == 2) {
           // the other half of the channels is in the peer CTA: swap partial sums
           const int slot = (ti & 1u) * 256 + sub * 128 + row;
@@ -852,13 +926,27 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
           lane_pass2(p, s, taddr, 0, p.BN, n0, valid, vox, vox2, rs);
       }
     }
-    if (!early) {
-      tc_fence_before();
-      mbar_arrive(smem_u32(&s.tempty[acc]));
-    }
+    if (!early) release(acc);
   }
 }
 
+// S = 2 throughout; narrow layers (and 1-row kernels) put a group's window and
+// weight tiles in one stage.
+template <bool PAIR>
+__device__ void run_mma(const ConvParams& p, const Smem& s, uint32_t tmem_base) {
+  if (p.kh_eff == 1)
+    mma_issuer<2, 1, 1, true, PAIR>(p, s, tmem_base);
+  else if (p.kh_eff == 2)
+    p.combined ? mma_issuer<2, 2, 2, true, PAIR>(p, s, tmem_base)
+               : mma_issuer<2, 2, 1, false, PAIR>(p, s, tmem_base);
+  else
+    p.combined ? mma_issuer<2, 3, 3, true, PAIR>(p, s, tmem_base)
+               : mma_issuer<2, 3, 1, false, PAIR>(p, s, tmem_base);
+}
+
+// PAIR (= p.pair) is a template parameter so that only the pair kernel holds
+// cta_group::2 instructions: a kernel with them is launched as clusters of 2.
+template <bool PAIR>
 __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_constant__ ConvParams p) {
   extern __shared__ uint8_t smem_raw[];
   const Smem s = carve(smem_raw, p);
@@ -875,7 +963,8 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&s.tfull[i]), 1);
-      mbar_init(smem_u32(&s.tempty[i]), 256);
+      // every epilogue thread releases the accumulator (both CTAs' with a pair)
+      mbar_init(smem_u32(&s.tempty[i]), PAIR ? 512 : 256);
     }
     mbar_init(smem_u32(s.drain), 1);
     mbar_init(smem_u32(&s.xbar[0]), 256);  // 256 epilogue threads of the peer CTA
@@ -894,8 +983,13 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
     }
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(s.tmem_slot), 512);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(s.tmem_slot), 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(s.tmem_slot), 512);
+      tmem_relinquish();
+    }
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&p.tmA);
@@ -903,39 +997,33 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
   }
   tc_fence_before();
   __syncthreads();
-  // With a CTA pair, both CTAs' barriers exist before either writes to the other.
-  if (p.nsplit == 2) cluster_sync_all();
+  // With a cluster of two, both CTAs' barriers exist before either writes to the other.
+  if (cluster2(p)) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *s.tmem_slot;
-  const int crank = p.nsplit == 2 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int crank = cluster2(p) ? static_cast<int>(cluster_ctarank()) : 0;
 
   if (warp == 0) {
-    if (lane == 0) producer(p, s, crank);
+    if (lane == 0) producer<PAIR>(p, s, crank);
   } else if (warp == 1) {
-    if (lane == 0) {
-      // S = 2 throughout; narrow layers (and 1-row kernels) put a group's
-      // window and weight tiles in one stage
-      if (p.kh_eff == 1)
-        mma_issuer<2, 1, 1, true>(p, s, tmem_base);
-      else if (p.kh_eff == 2)
-        p.combined ? mma_issuer<2, 2, 2, true>(p, s, tmem_base)
-                   : mma_issuer<2, 2, 1, false>(p, s, tmem_base);
-      else
-        p.combined ? mma_issuer<2, 3, 3, true>(p, s, tmem_base)
-                   : mma_issuer<2, 3, 1, false>(p, s, tmem_base);
-    }
+    // a pair's MMAs are rank 0's
+    if (lane == 0 && (!PAIR || crank == 0)) run_mma<PAIR>(p, s, tmem_base);
   } else {
-    epilogue(p, s, tmem_base, warp, lane, crank);
+    epilogue<PAIR>(p, s, tmem_base, warp, lane, crank);
   }
 
   tc_fence_before();
   __syncthreads();
-  // Neither CTA of a pair leaves while the other may still write into it.
-  if (p.nsplit == 2) cluster_sync_all();
+  // Neither CTA of a cluster leaves while the other may still write into it
+  // (or, with a pair, while rank 0's MMAs may still read its shared memory).
+  if (cluster2(p)) cluster_sync_all();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem_base, 512);
+    else
+      tmem_dealloc(tmem_base, 512);
   }
 }
 
@@ -982,7 +1070,7 @@ cudaLaunchConfig_t launch_config(const ConvParams& p, int grid, size_t smem, cud
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = p.nsplit == 2 ? 2 : 1;
+  attr[0].val.clusterDim.x = (p.nsplit == 2 || p.pair) ? 2 : 1;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
@@ -993,7 +1081,8 @@ cudaLaunchConfig_t launch_config(const ConvParams& p, int grid, size_t smem, cud
 
 int conv_tc_max_clusters(const ConvParams& p) {
   const size_t smem = launch_smem(p);
-  if (cudaFuncSetAttribute(conv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kern = p.pair ? conv_tc_kernel<true> : conv_tc_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess) {
     cudaGetLastError();
     return 0;
@@ -1001,7 +1090,7 @@ int conv_tc_max_clusters(const ConvParams& p) {
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = launch_config(p, 2, smem, nullptr, attr);
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, conv_tc_kernel, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -1010,12 +1099,13 @@ int conv_tc_max_clusters(const ConvParams& p) {
 
 cudaError_t launch_conv_tc(const ConvParams& p, int grid, cudaStream_t stream) {
   const size_t smem = launch_smem(p);
-  cudaError_t e = cudaFuncSetAttribute(conv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kern = p.pair ? conv_tc_kernel<true> : conv_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = launch_config(p, grid, smem, stream, attr);
-  e = cudaLaunchKernelEx(&cfg, conv_tc_kernel, p);
+  e = cudaLaunchKernelEx(&cfg, kern, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -61,6 +61,9 @@ struct ConvParams {
                      //    t -> 2t - 1 and 2t, frame 0 once; 2: t -> 2t and 2t + 1)
   int nsplit;        // 2: a cluster of 2 CTAs splits N (rank = N tile) and exchanges the
                      //    RMS partial sums over distributed shared memory
+  int pair;          // 1: a cluster of 2 CTAs shares M = 256 MMAs (cta_group::2): rank r
+                     //    takes M tile 2i + r of pair tile i and loads half of each weight
+                     //    tile (BN / 2 rows); rank 0 issues the MMAs
   int has_cache;
   int BN, n_tiles;
   int S;             // MMA sub-tiles per CTA tile (2)
@@ -92,8 +95,12 @@ __host__ __device__ inline uint32_t conv_tc_a_rows(const ConvParams& p) {
 __host__ __device__ inline uint32_t conv_tc_a_bytes(const ConvParams& p) {
   return (conv_tc_a_rows(p) * static_cast<uint32_t>(p.tile_cols) * 128u + 1023u) & ~1023u;
 }
+// Rows of one weight tile held by a CTA: BN, or BN / 2 with a CTA pair.
+__host__ __device__ inline int conv_tc_b_rows(const ConvParams& p) {
+  return p.pair ? p.BN / 2 : p.BN;
+}
 __host__ __device__ inline uint32_t conv_tc_b_bytes(const ConvParams& p) {
-  return static_cast<uint32_t>(p.b_tiles * p.nw * p.BN) * 128u;
+  return static_cast<uint32_t>(p.b_tiles * p.nw * conv_tc_b_rows(p)) * 128u;
 }
 // TMEM columns per sub-tile accumulator: the MMA's N (nw BN) rounded up to 32.
 __host__ __device__ inline uint32_t conv_tc_acc_stride(const ConvParams& p) {
