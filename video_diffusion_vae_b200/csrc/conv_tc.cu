@@ -31,13 +31,19 @@
 //   warps 2..9  epilogue, two groups of 4 warps (one warp per TMEM lane
 //               quarter each) taking alternate sub-tiles: one TMEM lane = one
 //               output voxel per thread.
-// The conv is bound by how fast L2 can refill shared memory, so the operand
-// bytes per MMA FLOP decide the speed: the row-tap windows load each input
-// row about once per (kt, kw) instead of once per tap.
+// The row-tap windows load each input row about once per (kt, kw) instead of
+// once per tap, which keeps the refill of shared memory from L2 off the
+// critical path.
 // 512 output channels with the next layer's norm fused: a cluster of two CTAs
 // splits N (each runs the S = 2, BN = 256 main loop on its half of the
 // channels for the same M tiles) and the two epilogues exchange each voxel's
 // partial sum of squares through distributed shared memory.
+// One N tile of 128 or 256 channels per CTA (no shortcut, not Winograd): a
+// cluster of two CTAs shares M = 256 MMAs (conv_tc_kernel<true>,
+// tcgen05.mma.cta_group::2): each CTA keeps its own tile and A windows and
+// loads half of every weight tile, rank 0 issues the MMAs and multicasts its
+// commits to both CTAs, and both epilogues release the accumulator on rank
+// 0's barrier.
 // tcgen05.mma issue runs nearly in step with execution, so every cycle the
 // issuing thread spends waiting on a barrier is a tensor-pipe bubble: S
 // sub-tiles per weight tile put S times more MMA work behind each wait.
