@@ -1050,6 +1050,17 @@ void conv_tc_choose_stages(ConvParams& p) {
     p.stages_a = p.stages_b = static_cast<int>(n < 2 ? 2 : n);
     return;
   }
+  // A pair's half weight tiles leave room for a third A window (measured:
+  // ~0.5-1 % on the 256-wide pair layers); otherwise two A stages
+  if (p.pair) {
+    size_t nb3 = (budget - 3 * a) / b;
+    if (nb3 > static_cast<size_t>(kMaxStages)) nb3 = kMaxStages;
+    if (nb3 >= 4) {
+      p.stages_a = 3;
+      p.stages_b = static_cast<int>(nb3);
+      return;
+    }
+  }
   // each A window serves kh_eff weight tiles: two A stages, the rest for B
   size_t nb = (budget - 2 * a) / b;
   if (nb > static_cast<size_t>(kMaxStages)) nb = kMaxStages;
