@@ -55,7 +55,9 @@ def test_pair_conv_two_n_tiles(T):
 
 @pytest.mark.parametrize("cin,cout,T,H,W", [(256, 128, 1, 5, 9), (256, 256, 3, 7, 11), (128, 256, 1, 16, 16)])
 def test_pair_upsample_conv(cin, cout, T, H, W):
-    """Upsample convs on pairs: partners share the phase (its 2 x 2 weights)."""
+    """Upsample convs on pairs: partners share the phase (its 2 x 2 weights).
+    These run the staged-store kernel (each warp's 32-channel chunks written
+    with TMA stores of 16-voxel row segments; the ragged widths clip at W)."""
     g = torch.Generator().manual_seed(cin + cout + T)
     x = synth.normal(g, (cin, T, H, W))
     w, b = synth.conv_params(g, cout, cin, 1, 3, 3)

@@ -139,6 +139,22 @@ bool encode_planes(CUtensorMap* m, const void* base, int C, int W, int H, int T,
          CUDA_SUCCESS;
 }
 
+// An epilogue output [rows][W][Q][C] (C channels, Q column phases) for staged
+// TMA stores of 32 channels x 16 voxels of one row: fp32 rows of 128 B under
+// the 128B swizzle, bf16 rows of 64 B under the 64B swizzle.
+bool encode_store(CUtensorMap* m, void* base, int eb, int C, int Q, int W, long rows) {
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(Q),
+                        static_cast<cuuint64_t>(W), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(C) * eb, static_cast<cuuint64_t>(C) * eb * Q,
+                           static_cast<cuuint64_t>(C) * eb * Q * W};
+  cuuint32_t box[4] = {32, 1, 16, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return g_encode(m, eb == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                  base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  eb == 4 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode_weights(CUtensorMap* m, const void* base, int K, int N, int box_rows,
                     CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N)};
@@ -262,7 +278,21 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   // with the column taps in N the two edge columns of a tile only feed their
   // neighbours: 16 computed columns give 14 outputs
   p.out_cols = kwn ? p.tile_cols - 2 : p.tile_cols;
+  // Staged TMA stores of the raw output and the activation (see conv_tc.cu) for
+  // the upsample convs on CTA pairs, whose outputs (four phases, fp32 + bf16)
+  // are large against their MMA work: there the per-lane stores kept the
+  // load/store pipe busy for 70 % of the kernel's time.  Elsewhere the buffers'
+  // 32 KB of shared memory (a ring stage less) cost more than they saved.
+  p.tma_out = (p.phases == 4 && p.pair && p.nw == 1 && !a.wino && a.ep.video == nullptr &&
+               !a.ep.out_f16 && p.BN % 32 == 0 && a.cout % 16 == 0 &&
+               (a.ep.out != nullptr || a.ep.act != nullptr) && a16(a.ep.out) && a16(a.ep.act))
+                  ? 1
+                  : 0;
   conv_tc_choose_stages(p);
+  if (p.tma_out && (p.combined ? p.stages_a < 3 : p.stages_b < 3)) {
+    p.tma_out = 0;
+    conv_tc_choose_stages(p);
+  }
   p.tiles_w = (a.W + p.out_cols - 1) / p.out_cols;
   p.tiles_h = (a.H + p.tile_rows - 1) / p.tile_rows;
   p.m_tiles = a.T * p.tiles_h * p.tiles_w;
@@ -291,6 +321,18 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
     if (!encode_act(&p.tmA, a.x, a.cin_pad, a.W, a.H, a.T, p.tile_cols, a_rows))
       return WVAE_ERR_CUDA;
     if (!encode_weights(&p.tmB, a.packed, L.taps * a.cin_pad, L.cout_pad, box_rows))
+      return WVAE_ERR_CUDA;
+  }
+  if (p.tma_out) {
+    // output frames (temporal 2x copies in phase mode) x rows per output frame
+    const int t_out = p.tdup == 1 ? 2 * a.T - 1 : (p.tdup == 2 ? 2 * a.T : a.T);
+    const int rows = a.phases == 4 ? (p.out_rows > 0 ? p.out_rows : 2 * a.H) : a.H;
+    const int q = a.phases == 4 ? 2 : 1;
+    if (a.ep.out != nullptr && !encode_store(&p.tmO, a.ep.out, a.ep.out_f32 ? 4 : 2, a.cout, q, a.W,
+                                             static_cast<long>(t_out) * rows))
+      return WVAE_ERR_CUDA;
+    if (a.ep.act != nullptr && !encode_store(&p.tmAct, a.ep.act, 2, a.cout, q, a.W,
+                                             static_cast<long>(t_out) * rows))
       return WVAE_ERR_CUDA;
   }
   if (a.cache != nullptr && !encode_act(&p.tmC, a.cache, a.cin_pad, a.W, a.H, a.KT - 1, p.tile_cols,

@@ -47,6 +47,12 @@
 // tcgen05.mma issue runs nearly in step with execution, so every cycle the
 // issuing thread spends waiting on a barrier is a tensor-pipe bubble: S
 // sub-tiles per weight tile put S times more MMA work behind each wait.
+// The upsample convs on CTA pairs (conv_tc_staged_kernel) write their outputs
+// through shared memory: each epilogue warp stages a 32-channel chunk of its 32
+// voxels in a 4 KB buffer and one lane issues TMA stores of its two 16-voxel
+// row segments, where per-lane stores of voxel rows kept the load/store pipe
+// busy for 70 % of these kernels' time (their four phases write fp32 + bf16
+// outputs four times the input's size).
 // The epilogue adds bias (and residual), and may emit the raw result (fp32 or
 // bf16, optionally 2x-upsampled), the next layer's SiLU(norm(.)) activation
 // (the whole channel vector of the voxel is in the thread's TMEM lane, so the
@@ -63,6 +69,7 @@ namespace {
 struct Smem {
   uint8_t* a_ring;        // A stage i at a_ring + i * a_bytes, 1024-aligned
   uint8_t* b_ring;        // B stage j at b_ring + j * b_bytes, 1024-aligned
+  uint32_t stage;         // staged-store buffers (tma_out): kStageWarpBytes per epilogue warp
   uint32_t a_bytes, b_bytes;
   uint64_t* full_a;       // [kMaxStages]
   uint64_t* empty_a;      // [kMaxStages]
@@ -91,7 +98,9 @@ __device__ __forceinline__ Smem carve(uint8_t* raw, const ConvParams& p) {
   s.b_bytes = conv_tc_b_bytes(p);
   s.a_ring = al;
   s.b_ring = al + p.stages_a * s.a_bytes;
-  uint8_t* ctrl = s.b_ring + p.stages_b * s.b_bytes;
+  uint8_t* stage = s.b_ring + p.stages_b * s.b_bytes;  // 1024-aligned: whole 1 KB stages
+  s.stage = smem_u32(stage);
+  uint8_t* ctrl = stage + conv_tc_stage_bytes(p);
   s.full_a = reinterpret_cast<uint64_t*>(ctrl);
   s.empty_a = s.full_a + kMaxStages;
   s.full_b = s.empty_a + kMaxStages;
@@ -562,6 +571,92 @@ __device__ __forceinline__ void store_f32(float* dst, const float (&v)[NC], bool
   for (int q = 0; q < NC / 4; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
 }
 
+// ---- staged stores (tma_out)
+// A warp's 32 voxels (one per lane) x 32 channels go through the warp's own
+// shared buffer, one row per voxel (fp32 rows of 128 B, bf16 rows of 64 B)
+// with the 16-byte pieces XOR-swizzled where the tensor map's 128B / 64B
+// swizzle expects them, so each 16-byte shared store of 8 lanes covers all 32
+// banks once.  Lane 0 then writes the two 16-voxel halves (each inside one
+// tile row) with one TMA store each.  Per-lane global stores of voxel rows
+// touch 32 cache lines per warp instruction, and on the layers with large
+// outputs they kept the load/store pipe busy for most of the kernel's time.
+struct StoreRows {  // this lane's voxel as a box origin (lanes 0 and 16 are read)
+  int ok;           // written: own tile, inside H x W and inside the row window
+  int q;            // column phase (phase mode), else 0
+  int w, r, r2;     // box coordinates: column, row of the [rows][W] view, and the
+                    // row of the second output frame (temporal 2x copies) or -1
+};
+
+struct Stage {
+  uint32_t buf;  // this warp's buffer
+  int lane;
+  StoreRows sr;
+};
+
+// The buffer is free once the previous chunk's bulk stores have read it.  (A
+// second buffer per warp, so that this waits on the chunk before that, measured
+// no faster: the wait is not what holds the epilogue up.)
+__device__ __forceinline__ void stage_acquire(const Stage& st) {
+  if (st.lane == 0) bulk_wait_read_all();
+  __syncwarp();
+}
+
+__device__ __forceinline__ void stage_f32(const Stage& st, const float (&v)[32]) {
+  const uint32_t row = st.buf + static_cast<uint32_t>(st.lane) * 128u;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    st_shared_v4(row + (static_cast<uint32_t>((j ^ st.lane) & 7) << 4), __float_as_uint(v[4 * j]),
+                 __float_as_uint(v[4 * j + 1]), __float_as_uint(v[4 * j + 2]),
+                 __float_as_uint(v[4 * j + 3]));
+}
+
+__device__ __forceinline__ void stage_b16(const Stage& st, const uint32_t (&u)[16]) {
+  const uint32_t row = st.buf + static_cast<uint32_t>(st.lane) * 64u;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    st_shared_v4(row + (static_cast<uint32_t>((j ^ (st.lane >> 1)) & 3) << 4), u[4 * j],
+                 u[4 * j + 1], u[4 * j + 2], u[4 * j + 3]);
+}
+
+// seg_bytes: bytes of 16 staged rows (2048 fp32, 1024 bf16); x: the first channel.
+__device__ __forceinline__ void stage_commit(const Stage& st, const CUtensorMap* tm,
+                                             uint32_t seg_bytes, int x) {
+  fence_proxy_async_smem();  // this lane's shared stores before the async proxy reads them
+  __syncwarp();
+  const StoreRows& a = st.sr;
+  const int ok1 = __shfl_sync(0xffffffffu, a.ok, 16);
+  const int w1 = __shfl_sync(0xffffffffu, a.w, 16);
+  const int r1 = __shfl_sync(0xffffffffu, a.r, 16);
+  const int rr1 = __shfl_sync(0xffffffffu, a.r2, 16);
+  if (st.lane == 0) {
+    if (a.ok) {
+      tma_store_4d(tm, st.buf, x, a.q, a.w, a.r);
+      if (a.r2 >= 0) tma_store_4d(tm, st.buf, x, a.q, a.w, a.r2);
+    }
+    if (ok1) {
+      tma_store_4d(tm, st.buf + seg_bytes, x, a.q, w1, r1);
+      if (rr1 >= 0) tma_store_4d(tm, st.buf + seg_bytes, x, a.q, w1, rr1);
+    }
+    bulk_commit_group();
+  }
+}
+
+// The raw result chunk (fp32 or bf16) through the buffer.
+__device__ __forceinline__ void stage_raw(const ConvParams& p, Stage& st, int x,
+                                          const float (&v)[32]) {
+  stage_acquire(st);
+  if (p.ep.out_f32) {
+    stage_f32(st, v);
+    stage_commit(st, &p.tmO, 2048, x);
+  } else {
+    uint32_t u[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) u[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+    stage_b16(st, u);
+    stage_commit(st, &p.tmO, 1024, x);
+  }
+}
+
 // Loads columns [c0, c0 + NC) of this thread's accumulator lane and returns
 // acc + bias (+ residual) in v.
 template <int NC>
@@ -593,6 +688,23 @@ __device__ __forceinline__ void store_raw(const ConvParams& p, int c0, int n0, s
       store_f16<NC>(static_cast<__half*>(ep.out) + off, v);
     else
       store_bf16<NC>(static_cast<__nv_bfloat16*>(ep.out) + off, v, ep.vec32 != 0);
+  }
+}
+
+// The next layer's activation bf16 pairs: SiLU_half((v rs) gamma/2 + beta/2).
+template <int NC>
+__device__ __forceinline__ void act_words(const ConvParams& p, const Smem& s, int c0, int n0,
+                                          float rs, const float (&v)[NC], uint32_t (&u)[NC / 2]) {
+  const float2 r2 = make_float2(rs, rs);
+  const float4* g4 = reinterpret_cast<const float4*>(s.gamma + n0 + c0);
+  const float4* b4 = reinterpret_cast<const float4*>(s.beta + n0 + c0);
+#pragma unroll
+  for (int e = 0; e < NC / 2; ++e) {  // channel pair e as two lanes of a 128-bit load
+    const float4 g = g4[e >> 1], b = b4[e >> 1];
+    const float2 g2 = (e & 1) ? make_float2(g.z, g.w) : make_float2(g.x, g.y);
+    const float2 b2 = (e & 1) ? make_float2(b.z, b.w) : make_float2(b.x, b.y);
+    const float2 o = silu_half2(ffma2(fmul2(make_float2(v[2 * e], v[2 * e + 1]), r2), g2, b2));
+    u[e] = pack_bf16x2(o.x, o.y);
   }
 }
 
@@ -642,6 +754,16 @@ __device__ __forceinline__ void store_act(const ConvParams& p, const Smem& s, in
   }
 }
 
+// The activation chunk through the buffer.
+__device__ __forceinline__ void stage_act(const ConvParams& p, const Smem& s, Stage& st,
+                                          int c0, int n0, float rs, const float (&v)[32]) {
+  uint32_t u[16];
+  act_words<32>(p, s, c0, n0, rs, v, u);
+  stage_acquire(st);
+  stage_b16(st, u);
+  stage_commit(st, &p.tmAct, 1024, n0 + c0);
+}
+
 // Outputs that need no RMS statistic: the raw result and the video.
 template <int NC>
 __device__ __forceinline__ void emit_chunk(const ConvParams& p, int c0, int n0,
@@ -682,10 +804,10 @@ __device__ __forceinline__ void tmem_store_chunk(uint32_t taddr, const float (&v
 // No second output voxel (see the temporal 2x copies in epilogue()).
 constexpr size_t kNoVox = ~static_cast<size_t>(0);
 
-template <int NC>
-__device__ __forceinline__ void pass1_chunk(const ConvParams& p, const Smem& s, uint32_t taddr,
-                                            int c0, int n0, bool valid, size_t vox, size_t vox2,
-                                            float& ss, bool keep) {
+template <int NC, bool STAGED>
+__device__ __forceinline__ void pass1_chunk(const ConvParams& p, const Smem& s, Stage& st,
+                                            uint32_t taddr, int c0, int n0, bool valid,
+                                            size_t vox, size_t vox2, float& ss, bool keep) {
   float v[NC];
   result_chunk<NC>(p, s, taddr, c0, n0, valid, vox, v);
   float2 sa = make_float2(0.0f, 0.0f), sb = sa;  // two packed chains
@@ -696,6 +818,11 @@ __device__ __forceinline__ void pass1_chunk(const ConvParams& p, const Smem& s, 
     sb = ffma2(x1, x1, sb);
   }
   ss += (sa.x + sa.y) + (sb.x + sb.y);
+  if constexpr (STAGED && NC == 32) {
+    if (p.ep.out != nullptr && n0 + c0 < p.cout) stage_raw(p, st, n0 + c0, v);
+    if (keep) tmem_store_chunk<NC>(taddr + c0, v);
+    return;
+  }
   if (valid) {
     store_raw<NC>(p, c0, n0, vox, v);
     if (vox2 != kNoVox) store_raw<NC>(p, c0, n0, vox2, v);
@@ -704,27 +831,34 @@ __device__ __forceinline__ void pass1_chunk(const ConvParams& p, const Smem& s, 
 }
 // keep = false: h is not stored back (the caller re-reads it from the fp32
 // raw output instead).
-__device__ __forceinline__ float lane_pass1(const ConvParams& p, const Smem& s, uint32_t taddr,
-                                           int c_lo, int c_hi, int n0, bool valid, size_t vox,
-                                           size_t vox2, bool keep) {
+template <bool STAGED>
+__device__ __forceinline__ float lane_pass1(const ConvParams& p, const Smem& s, Stage& st,
+                                           uint32_t taddr, int c_lo, int c_hi, int n0,
+                                           bool valid, size_t vox, size_t vox2, bool keep) {
   float ss = 0.0f;
   int c0 = c_lo;
-  for (; c0 + 32 <= c_hi; c0 += 32) pass1_chunk<32>(p, s, taddr, c0, n0, valid, vox, vox2, ss, keep);
-  if (c0 < c_hi) pass1_chunk<16>(p, s, taddr, c0, n0, valid, vox, vox2, ss, keep);
+  for (; c0 + 32 <= c_hi; c0 += 32)
+    pass1_chunk<32, STAGED>(p, s, st, taddr, c0, n0, valid, vox, vox2, ss, keep);
+  if (c0 < c_hi) pass1_chunk<16, STAGED>(p, s, st, taddr, c0, n0, valid, vox, vox2, ss, keep);
   if (keep) tmem_wait_st();
   return ss;
 }
 
 // Second pass reading h back from the fp32 raw output this thread wrote in
 // pass 1 (the accumulator is released already).
-__device__ __forceinline__ void lane_pass2_global(const ConvParams& p, const Smem& s, int n0,
-                                                 bool valid, size_t vox, size_t vox2, float rs) {
-  if (!valid) return;
+template <bool STAGED>
+__device__ __forceinline__ void lane_pass2_global(const ConvParams& p, const Smem& s,
+                                                 Stage& st, int n0, bool valid, size_t vox,
+                                                 size_t vox2, float rs) {
+  if (!STAGED && !valid) return;
   const float* h = static_cast<const float*>(p.ep.out) + vox * p.cout + n0;
   int c0 = 0;
   for (; c0 + 32 <= p.BN; c0 += 32) {
     float v[32];
-    if (p.ep.vec32) {
+    if (!valid) {  // staged stores: the warp's lanes all take part
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+    } else if (p.ep.vec32) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t u[8];
@@ -743,10 +877,14 @@ __device__ __forceinline__ void lane_pass2_global(const ConvParams& p, const Sme
         v[4 * q + 3] = f.w;
       }
     }
+    if constexpr (STAGED) {
+      if (n0 + c0 < p.cout) stage_act(p, s, st, c0, n0, rs, v);
+      continue;
+    }
     store_act<32>(p, s, c0, n0, vox, rs, v);
     if (vox2 != kNoVox) store_act<32>(p, s, c0, n0, vox2, rs, v);
   }
-  if (c0 < p.BN) {
+  if (c0 < p.BN && valid) {
     float v[16];
     const float4* h4 = reinterpret_cast<const float4*>(h + c0);
 #pragma unroll
@@ -763,14 +901,17 @@ __device__ __forceinline__ void lane_pass2_global(const ConvParams& p, const Sme
 }
 
 // Second pass: the next layer's activation SiLU(h r gamma + beta) from h in the lane.
-__device__ __forceinline__ void lane_pass2(const ConvParams& p, const Smem& s, uint32_t taddr,
-                                          int c_lo, int c_hi, int n0, bool valid, size_t vox,
-                                          size_t vox2, float rs) {
+template <bool STAGED>
+__device__ __forceinline__ void lane_pass2(const ConvParams& p, const Smem& s, Stage& st,
+                                          uint32_t taddr, int c_lo, int c_hi, int n0, bool valid,
+                                          size_t vox, size_t vox2, float rs) {
   int c0 = c_lo;
   for (; c0 + 32 <= c_hi; c0 += 32) {
     float v[32];
     tmem_load_chunk<32>(taddr + c0, v);
-    if (valid) {
+    if constexpr (STAGED) {
+      if (n0 + c0 < p.cout) stage_act(p, s, st, c0, n0, rs, v);
+    } else if (valid) {
       store_act<32>(p, s, c0, n0, vox, rs, v);
       if (vox2 != kNoVox) store_act<32>(p, s, c0, n0, vox2, rs, v);
     }
@@ -786,14 +927,18 @@ __device__ __forceinline__ void lane_pass2(const ConvParams& p, const Smem& s, u
 }
 
 // Single pass when no norm is fused: raw result and / or video.
-__device__ __forceinline__ void lane_emit(const ConvParams& p, const Smem& s, uint32_t taddr,
-                                          int c_lo, int c_hi, int n0, bool valid, size_t vox,
-                                          size_t vox2, const TileCoord& tc, int h, int w) {
+template <bool STAGED>
+__device__ __forceinline__ void lane_emit(const ConvParams& p, const Smem& s, Stage& st,
+                                          uint32_t taddr, int c_lo, int c_hi, int n0, bool valid,
+                                          size_t vox, size_t vox2, const TileCoord& tc, int h,
+                                          int w) {
   int c0 = c_lo;
   for (; c0 + 32 <= c_hi; c0 += 32) {
     float v[32];
     result_chunk<32>(p, s, taddr, c0, n0, valid, vox, v);
-    if (valid) {
+    if constexpr (STAGED) {  // no video with staged stores
+      if (p.ep.out != nullptr && n0 + c0 < p.cout) stage_raw(p, st, n0 + c0, v);
+    } else if (valid) {
       emit_chunk<32>(p, c0, n0, tc, h, w, vox, v);
       if (vox2 != kNoVox) store_raw<32>(p, c0, n0, vox2, v);
     }
@@ -829,7 +974,7 @@ __device__ __noinline__ void lane_emit_taps_in_n(const ConvParams& p, const Smem
   if (valid) emit_chunk<NB>(p, 0, n0, tc, h, w, vox, v);
 }
 
-template <bool PAIR>
+template <bool PAIR, bool STAGED>
 __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base, int warp,
                          int lane, int crank) {
   const int q = warp & 3;           // TMEM lane quarter this warp may access
@@ -842,6 +987,9 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
   // accumulator fills TMEM and CTAs run several tiles).
   const bool early = p.early_release != 0;
   uint32_t ti = 0;
+  Stage st;
+  st.buf = s.stage + static_cast<uint32_t>(warp - 2) * kStageWarpBytes;
+  st.lane = lane;
   // The accumulator's release: on this CTA's barrier, or on rank 0's with a
   // pair (rank 0's MMAs write both CTAs' accumulators).
   auto release = [&](uint32_t acc) {
@@ -898,15 +1046,24 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
       };
       const size_t vox = out_vox(t0);
       const size_t vox2 = t1 < 0 ? kNoVox : out_vox(t1);
+      st.sr.ok = valid ? 1 : 0;
+      st.sr.q = p.phases == 4 ? (tc.phase & 1) : 0;
+      st.sr.w = w;
+      {
+        const int hr = p.phases == 4 ? ho : h;     // row inside the output frame
+        const int rows = p.phases == 4 ? Ho : p.H;  // rows per output frame
+        st.sr.r = t0 * rows + hr;
+        st.sr.r2 = t1 < 0 ? -1 : t1 * rows + hr;
+      }
       const uint32_t n_stride = conv_tc_acc_stride(p);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              (acc * static_cast<uint32_t>(p.S) + static_cast<uint32_t>(sub)) * n_stride;
       if (p.nw > 1) {
         lane_emit_taps_in_n<16>(p, s, taddr, n0, valid, vox, tc, h, w);  // BN = 16
       } else if (p.ep.act == nullptr) {
-        lane_emit(p, s, taddr, 0, p.BN, n0, valid, vox, vox2, tc, h, w);
+        lane_emit<STAGED>(p, s, st, taddr, 0, p.BN, n0, valid, vox, vox2, tc, h, w);
       } else {
-        float ss = lane_pass1(p, s, taddr, 0, p.BN, n0, valid, vox, vox2, !early);
+        float ss = lane_pass1<STAGED>(p, s, st, taddr, 0, p.BN, n0, valid, vox, vox2, !early);
         if (early) release(acc);
         if (p.nsplit == 2) {
           // the other half of the channels is in the peer CTA: swap partial sums
@@ -921,19 +1078,34 @@ __device__ void epilogue(const ConvParams& p, const Smem& s, uint32_t tmem_base,
                       ? 1
                       : 0;
           got = __shfl_sync(0xffffffffu, got, 0);
-          if (!got) return;
+          if (!got) {
+            if (STAGED && lane == 0) bulk_wait_all();
+            return;
+          }
           __syncwarp();
           ss += s.xpart[slot];
         }
         const float rs = rootC / fmaxf(sqrtf(ss), p.ep.eps);
-        if (early)
-          lane_pass2_global(p, s, n0, valid, vox, vox2, rs);
-        else
-          lane_pass2(p, s, taddr, 0, p.BN, n0, valid, vox, vox2, rs);
+        if (early) {
+          if constexpr (STAGED) {
+            // pass 2 reads h back from the raw output that lane 0's bulk stores wrote
+            if (lane == 0) {
+              bulk_wait_all();
+              fence_proxy_async_global();
+            }
+            __syncwarp();
+            asm volatile("" ::: "memory");
+          }
+          lane_pass2_global<STAGED>(p, s, st, n0, valid, vox, vox2, rs);
+        } else {
+          lane_pass2<STAGED>(p, s, st, taddr, 0, p.BN, n0, valid, vox, vox2, rs);
+        }
       }
     }
     if (!early) release(acc);
   }
+  // the buffers' last bulk stores complete before the CTA leaves
+  if (STAGED && lane == 0) bulk_wait_all();
 }
 
 // S = 2 throughout; narrow layers (and 1-row kernels) put a group's window and
@@ -950,10 +1122,11 @@ __device__ void run_mma(const ConvParams& p, const Smem& s, uint32_t tmem_base) 
                : mma_issuer<2, 3, 1, false, PAIR>(p, s, tmem_base);
 }
 
-// PAIR (= p.pair) is a template parameter so that only the pair kernel holds
+// PAIR (= p.pair) is a template parameter so that only the pair kernels hold
 // cta_group::2 instructions: a kernel with them is launched as clusters of 2.
-template <bool PAIR>
-__global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_constant__ ConvParams p) {
+// STAGED (= p.tma_out) picks the epilogue's staged TMA stores.
+template <bool PAIR, bool STAGED>
+__device__ __forceinline__ void conv_tc_body(const ConvParams& p) {
   extern __shared__ uint8_t smem_raw[];
   const Smem s = carve(smem_raw, p);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -1015,7 +1188,7 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
     // a pair's MMAs are rank 0's
     if (lane == 0 && (!PAIR || crank == 0)) run_mma<PAIR>(p, s, tmem_base);
   } else {
-    epilogue<PAIR>(p, s, tmem_base, warp, lane, crank);
+    epilogue<PAIR, STAGED>(p, s, tmem_base, warp, lane, crank);
   }
 
   tc_fence_before();
@@ -1033,15 +1206,27 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
   }
 }
 
+template <bool PAIR>
+__global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_constant__ ConvParams p) {
+  conv_tc_body<PAIR, false>(p);
+}
+
+// The upsample convs on CTA pairs, their outputs written by staged TMA stores.
+__global__ void __launch_bounds__(kConvThreads, 1)
+    conv_tc_staged_kernel(const __grid_constant__ ConvParams p) {
+  conv_tc_body<true, true>(p);
+}
+
 }  // namespace
 
 size_t conv_tc_smem_bytes(const ConvParams& p) {
   return 1024 + static_cast<size_t>(p.stages_a) * conv_tc_a_bytes(p) +
-         static_cast<size_t>(p.stages_b) * conv_tc_b_bytes(p) + kCtrlBytes;
+         static_cast<size_t>(p.stages_b) * conv_tc_b_bytes(p) + conv_tc_stage_bytes(p) + kCtrlBytes;
 }
 
 void conv_tc_choose_stages(ConvParams& p) {
-  const size_t budget = 232448 - 1024 - kCtrlBytes;  // 227 KB opt-in per block
+  // 227 KB opt-in per block
+  const size_t budget = 232448 - 1024 - kCtrlBytes - conv_tc_stage_bytes(p);
   const size_t a = conv_tc_a_bytes(p), b = conv_tc_b_bytes(p);
   if (p.combined) {
     // one stage per group: equal depths
@@ -1098,7 +1283,7 @@ cudaLaunchConfig_t launch_config(const ConvParams& p, int grid, size_t smem, cud
 
 int conv_tc_max_clusters(const ConvParams& p) {
   const size_t smem = launch_smem(p);
-  auto kern = p.pair ? conv_tc_kernel<true> : conv_tc_kernel<false>;
+  auto kern = p.tma_out ? conv_tc_staged_kernel : (p.pair ? conv_tc_kernel<true> : conv_tc_kernel<false>);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess) {
     cudaGetLastError();
@@ -1116,7 +1301,7 @@ int conv_tc_max_clusters(const ConvParams& p) {
 
 cudaError_t launch_conv_tc(const ConvParams& p, int grid, cudaStream_t stream) {
   const size_t smem = launch_smem(p);
-  auto kern = p.pair ? conv_tc_kernel<true> : conv_tc_kernel<false>;
+  auto kern = p.tma_out ? conv_tc_staged_kernel : (p.pair ? conv_tc_kernel<true> : conv_tc_kernel<false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;

@@ -47,6 +47,10 @@ struct ConvParams {
   CUtensorMap tmA2;  // shortcut input, bf16 [T][H][W][cin2_pad], box {64, tile_cols,
                      // tile_rows, 1} (cin2_pad > 0)
   CUtensorMap tmB2;  // shortcut weights, bf16 [cout_pad][cin2_pad]
+  CUtensorMap tmO;   // staged stores (tma_out): the raw output viewed as [rows][W][Q][cout]
+                     // (Q = 2 column phases in phase mode, else 1; rows = output frames x
+                     // output rows), fp32 (128B swizzle) or bf16 (64B), box {32, 1, 16, 1}
+  CUtensorMap tmAct; // staged stores: the activation output, bf16, as tmO
   int T, H, W;
   int cin_pad, cin2_pad;
   int cout, cout_pad;
@@ -79,6 +83,9 @@ struct ConvParams {
                      // in one stage on one barrier (A and B rings in lockstep)
   int tiles_w, tiles_h, m_tiles, num_tiles;
   int stages_a, stages_b, num_acc;  // A-window ring, weight-tile ring, TMEM accumulators
+  int tma_out;       // 1: the epilogue stages 32-channel chunks in shared memory (a buffer
+                     //    per epilogue warp) and writes them with TMA stores (tmO / tmAct)
+                     //    instead of per-lane stores
   int early_release; // 1: release the accumulator after epilogue pass 1 (fused norm + fp32
                      //    raw output, one accumulator, several tiles per CTA)
   int groups_main;   // K groups of the main segment: (kt, column tap, 64 input channels)
@@ -105,6 +112,11 @@ __host__ __device__ inline uint32_t conv_tc_b_bytes(const ConvParams& p) {
 // TMEM columns per sub-tile accumulator: the MMA's N (nw BN) rounded up to 32.
 __host__ __device__ inline uint32_t conv_tc_acc_stride(const ConvParams& p) {
   return (static_cast<uint32_t>(p.nw * p.BN) + 31u) & ~31u;
+}
+// Staged-store buffers: 4 KB per epilogue warp (32 voxels x 32 fp32 channels).
+constexpr uint32_t kStageWarpBytes = 4096;
+__host__ __device__ inline uint32_t conv_tc_stage_bytes(const ConvParams& p) {
+  return p.tma_out ? 8u * kStageWarpBytes : 0u;
 }
 size_t conv_tc_smem_bytes(const ConvParams& p);
 // Sets p.stages_a / p.stages_b for the layer (needs BN, tile shape, kh_eff).
