@@ -278,13 +278,21 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
   // with the column taps in N the two edge columns of a tile only feed their
   // neighbours: 16 computed columns give 14 outputs
   p.out_cols = kwn ? p.tile_cols - 2 : p.tile_cols;
-  // Staged TMA stores of the raw output and the activation (see conv_tc.cu) for
-  // the upsample convs on CTA pairs, whose outputs (four phases, fp32 + bf16)
-  // are large against their MMA work: there the per-lane stores kept the
-  // load/store pipe busy for 70 % of the kernel's time.  Elsewhere the buffers'
-  // 32 KB of shared memory (a ring stage less) cost more than they saved.
-  p.tma_out = (p.phases == 4 && p.pair && p.nw == 1 && !a.wino && a.ep.video == nullptr &&
-               !a.ep.out_f16 && p.BN % 32 == 0 && a.cout % 16 == 0 &&
+  p.tiles_w = (a.W + p.out_cols - 1) / p.out_cols;
+  p.tiles_h = (a.H + p.tile_rows - 1) / p.tile_rows;
+  p.m_tiles = a.T * p.tiles_h * p.tiles_w;
+  p.num_tiles = p.m_tiles * per_m;
+  // Staged TMA stores of the raw output and the activation (see conv_tc.cu) on
+  // CTA pairs, for the upsample convs, whose outputs (four phases, fp32 + bf16)
+  // are large against their MMA work (the per-lane stores kept the load/store
+  // pipe busy for 70 % of the kernel's time), and for the layers whose one
+  // accumulator is released after epilogue pass 1 (fp32 + bf16 outputs, the
+  // next tile's MMAs waiting on that pass).  Elsewhere the buffers' 32 KB of
+  // shared memory (a ring stage less) cost more than they saved.
+  const bool early_layer = p.num_acc == 1 && a.ep.act != nullptr && a.ep.out != nullptr &&
+                           a.ep.out_f32 && p.num_tiles > slots;
+  p.tma_out = (p.pair && (p.phases == 4 || early_layer) && p.nw == 1 && !a.wino &&
+               a.ep.video == nullptr && !a.ep.out_f16 && p.BN % 32 == 0 && a.cout % 16 == 0 &&
                (a.ep.out != nullptr || a.ep.act != nullptr) && a16(a.ep.out) && a16(a.ep.act))
                   ? 1
                   : 0;
@@ -293,10 +301,6 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
     p.tma_out = 0;
     conv_tc_choose_stages(p);
   }
-  p.tiles_w = (a.W + p.out_cols - 1) / p.out_cols;
-  p.tiles_h = (a.H + p.tile_rows - 1) / p.tile_rows;
-  p.m_tiles = a.T * p.tiles_h * p.tiles_w;
-  p.num_tiles = p.m_tiles * per_m;
   p.groups_main = (a.phases == 4 ? 1 : a.KT) * p.kw_eff * (a.cin_pad / kBK);
   p.groups = p.groups_main + a.cin2_pad / kBK;
   a.ep.bias = reinterpret_cast<const float*>(static_cast<const char*>(a.packed) + L.bias_off);
@@ -342,10 +346,7 @@ wvae_status run_tc_conv(const DeviceInfo& d, TcConv a, cudaStream_t stream) {
     if (!encode_act(&p.tmA2, a.x2, a.cin2_pad, a.W, a.H, a.T, p.tile_cols, p.tile_rows)) return WVAE_ERR_CUDA;
     if (!encode_weights(&p.tmB2, a.packed2, a.cin2_pad, L.cout_pad, box_rows)) return WVAE_ERR_CUDA;
   }
-  p.early_release = (p.num_acc == 1 && a.ep.act != nullptr && a.ep.out != nullptr &&
-                     a.ep.out_f32 && p.num_tiles > slots)
-                        ? 1
-                        : 0;
+  p.early_release = early_layer ? 1 : 0;
   int grid;
   if (p.nsplit == 2 || p.pair) {
     int clusters = conv_tc_max_clusters(p);

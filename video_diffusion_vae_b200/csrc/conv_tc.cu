@@ -47,12 +47,13 @@
 // tcgen05.mma issue runs nearly in step with execution, so every cycle the
 // issuing thread spends waiting on a barrier is a tensor-pipe bubble: S
 // sub-tiles per weight tile put S times more MMA work behind each wait.
-// The upsample convs on CTA pairs (conv_tc_staged_kernel) write their outputs
+// The upsample convs on CTA pairs and the pair layers whose one accumulator is
+// released after epilogue pass 1 (conv_tc_staged_kernel) write their outputs
 // through shared memory: each epilogue warp stages a 32-channel chunk of its 32
 // voxels in a 4 KB buffer and one lane issues TMA stores of its two 16-voxel
 // row segments, where per-lane stores of voxel rows kept the load/store pipe
-// busy for 70 % of these kernels' time (their four phases write fp32 + bf16
-// outputs four times the input's size).
+// busy for 70 % of the upsample convs' time (their four phases write fp32 +
+// bf16 outputs four times the input's size).
 // The epilogue adds bias (and residual), and may emit the raw result (fp32 or
 // bf16, optionally 2x-upsampled), the next layer's SiLU(norm(.)) activation
 // (the whole channel vector of the voxel is in the thread's TMEM lane, so the
@@ -1211,7 +1212,7 @@ __global__ void __launch_bounds__(kConvThreads, 1) conv_tc_kernel(const __grid_c
   conv_tc_body<PAIR, false>(p);
 }
 
-// The upsample convs on CTA pairs, their outputs written by staged TMA stores.
+// The pair kernel whose epilogue writes its outputs with staged TMA stores.
 __global__ void __launch_bounds__(kConvThreads, 1)
     conv_tc_staged_kernel(const __grid_constant__ ConvParams p) {
   conv_tc_body<true, true>(p);
