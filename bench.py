@@ -760,7 +760,7 @@ def main():
             "config": bench_config(world, args.split),
             "tflops": sum(f for _, f in layers) * args.steps / (total_ms * 1e-3) / 1e12,
             "roofline": {"bound": "tensor",
-                         "kernel": "the 21 conv launches of a step: conv_tc_kernel x 20, head_tc_kernel x 1",
+                         "kernel": "the 21 conv launches of a step: conv_tc_kernel / conv_tc_staged_kernel x 20 (one body), head_tc_kernel x 1",
                          "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
                          "frac": achieved / peak_t,
                          "peak_kind": f"{peak_kind} bf16 burst (sub-millisecond launches)",
